@@ -1,0 +1,171 @@
+/*
+ * libmla -- MLA (Multi-head Latent Attention) prefill attention for NVIDIA
+ * B200 (sm_100a).  C ABI: plain pointers and sizes, no framework types.
+ *
+ * What the calls compute (sources named by page and section):
+ *
+ *   O = softmax(Q K^T * softmax_scale [+ causal mask]) V
+ *
+ * the only formula the pages print ("SparseFlashMla" README, Description --
+ * Formula, where K~ = V~ are the rows that take part), over ragged batches
+ * given by cu_seqlens_q / cu_seqlens_k ("Sgl project Sglang FA4 Interface",
+ * I/O Contract), with MLA head dims: Q/K have 128 nope + 64 rope = 192 dims,
+ * V has 128 (vLLM "flash_attn.py" MLA prefill backend,
+ * supports_mla_dimensions and FA4MLAPrefillKernel.dispatch), K/V already
+ * expanded to every head (same file, module comment: qhead_per_kvhead = 1).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory and keeps no pointer after return.
+ *   - Every call only enqueues work on `stream` (NULL = legacy default
+ *     stream) and returns; there is no host synchronisation and no
+ *     device-to-host copy.  Outputs are valid once the stream reaches the
+ *     point after the call.
+ *   - bf16 tensors are packed and row-major exactly as described per call;
+ *     tensors read by TMA (q, k, v, kv_latent) need 16-byte aligned bases.
+ *   - Errors: the return value is an mla_status.  Host-checkable problems
+ *     (null or misaligned pointers, bad sizes, unsupported GPU) are reported
+ *     before anything is launched.  Device-resident metadata (cu_seqlens
+ *     values, index values) is not validated; out-of-range sparse indices
+ *     are treated as padding by the kernel.  Kernel waits are bounded: a
+ *     wait that gives up sets a bit in the device status word (see
+ *     mla_device_status) instead of hanging.
+ *   - LSE ("log-sum-exp", float32 per the FA4 interface I/O Contract) is the
+ *     natural log of sum_j exp(softmax_scale * q.k_j), laid out [heads,
+ *     tokens]; a row that sees no key gets O = 0 and LSE = -inf.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL = default stream. */
+typedef struct CUstream_st* mla_stream_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or value  */
+  MLA_ERR_UNSUPPORTED = 2, /* not an sm_100 GPU, or an unsupported shape   */
+  MLA_ERR_CUDA = 3         /* a CUDA runtime/driver call or launch failed  */
+} mla_status;
+
+/* Bits of the device status word. */
+#define MLA_DEVSTAT_WAIT_TIMEOUT_LOAD 0x1u    /* load warp gave up waiting    */
+#define MLA_DEVSTAT_WAIT_TIMEOUT_MMA 0x2u     /* MMA warp gave up waiting     */
+#define MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX 0x4u /* softmax warps gave up waiting */
+#define MLA_DEVSTAT_WAIT_TIMEOUT_TEST 0x100u  /* mla_debug_wait_timeout probe  */
+
+/* Human-readable text for an mla_status value (static storage). */
+const char* mla_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int mla_version(void);
+
+/*
+ * Dense varlen MLA prefill forward.
+ *
+ * Computes, for every sequence b, head h and query row i of b,
+ *   O[i,h,:]  = sum_j softmax_j(softmax_scale * q[i,h,:].k[j,h,:]) v[j,h,:]
+ *   lse[h,i]  = ln sum_j exp(softmax_scale * q[i,h,:].k[j,h,:])
+ * over the keys j of sequence b that row i may see: all Lk keys when
+ * causal == 0; keys j <= i + (Lk - Lq) when causal != 0 (bottom-right
+ * aligned; equal to j <= i when Lq == Lk, the new-token case of the vLLM
+ * backend's run_prefill_new_tokens; causal == 0 with a separate key set is
+ * its run_prefill_context_chunk).
+ *
+ * Arguments:
+ *   q            bf16 [total_q, num_heads, 192], contiguous, 16-B aligned.
+ *   k            bf16 [total_k, num_heads, 192], contiguous, 16-B aligned.
+ *   v            bf16 [total_k, num_heads, 128], contiguous, 16-B aligned.
+ *   cu_seqlens_q int32 [batch+1] on the device: cu[0] = 0, non-decreasing,
+ *                cu[batch] = total_q.  Sequence b owns query rows
+ *                [cu_q[b], cu_q[b+1]).
+ *   cu_seqlens_k int32 [batch+1] on the device, same rules for keys.
+ *   max_seqlen_q upper bound on cu_q[b+1] - cu_q[b] (rows past it are not
+ *                computed); max_seqlen_k likewise for keys (informational).
+ *   softmax_scale finite, > 0; multiplies q.k (1/sqrt(192) for MLA).
+ *   causal       0 or 1.
+ *   out          bf16 [total_q, num_heads, 128], 16-B aligned; fully written.
+ *   lse          float32 [num_heads, total_q] or NULL (not returned).
+ *   stream       stream to enqueue on.
+ *   batch, num_heads, total_q, total_k: sizes (total_* >= 0, batch >= 1,
+ *                1 <= num_heads <= 65535, batch <= 65535).
+ * Returns MLA_OK or an error; on error nothing was launched.
+ */
+int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+                    float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
+                    int batch, int num_heads, int total_q, int total_k);
+
+/*
+ * Merge two partial attention results over disjoint key sets A and B into
+ * the result over A u B (the context-chunk + new-token combination of the
+ * vLLM MLA prefill backend; the same log-sum-exp identity as the split-KV
+ * combine kernels named on the FA4 interface page and the Mojo mla module):
+ *   lse  = m + ln(exp(lse_a - m) + exp(lse_b - m)),  m = max(lse_a, lse_b)
+ *   out  = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b
+ * A side with lse = -inf has weight 0; if both are -inf, out = 0 and
+ * lse = -inf.
+ *
+ *   o_a, o_b, out     bf16 [num_tokens, num_heads, head_dim], 16-B aligned;
+ *                     out may be the same pointer as o_a or o_b.
+ *   lse_a, lse_b      float32 [num_heads, num_tokens].
+ *   lse_out           float32 [num_heads, num_tokens] or NULL; must not
+ *                     overlap lse_a or lse_b (MLA_ERR_INVALID_ARG if it is
+ *                     the same pointer).
+ *   head_dim          a positive multiple of 8.
+ */
+int mla_attn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                   void* out, float* lse_out, int num_tokens, int num_heads, int head_dim,
+                   mla_stream_t stream);
+
+/*
+ * Absorbed top-k sparse MLA prefill forward ("SparseFlashMla" README,
+ * Formula with K~ = V~; Parameters: index -1 = invalid or padded slot;
+ * Constraints: indices [Q_T, KV_N = 1, K], one list per token shared by all
+ * heads; Mojo "mla_prefill_branch_sparse_fp8": the absorbed sparse prefill
+ * over the BF16 latent cache with indices already mapped to physical rows).
+ *
+ * For token t and head h, with R(t) = { r : 0 <= indices[t,r] < num_kv_rows }:
+ *   s_r       = softmax_scale * q[t,h,:] . kv_latent[indices[t,r], :]  (576 dims)
+ *   out[t,h,:] = sum_{r in R(t)} softmax_r(s) kv_latent[indices[t,r], 0:512]
+ *   lse[h,t]  = ln sum_{r in R(t)} exp(s_r)
+ *
+ *   q          bf16 [num_tokens, num_heads, 576] (512 latent + 64 rope).
+ *   kv_latent  bf16 [num_kv_rows, 576]; V is its first 512 dims.
+ *   indices    int32 [num_tokens, topk]; any value < 0 or >= num_kv_rows is
+ *              padding and is skipped.
+ *   out        bf16 [num_tokens, num_heads, 512].
+ *   lse        float32 [num_heads, num_tokens] or NULL.
+ *   softmax_scale finite, > 0 (1/sqrt(576) for the absorbed shape).
+ *   num_heads  1..128.
+ */
+int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* indices,
+                           int topk, float softmax_scale, void* out, float* lse,
+                           mla_stream_t stream, int num_tokens, int num_heads, int num_kv_rows);
+
+/*
+ * Read (and optionally clear) the device status word of the current device:
+ * the OR of MLA_DEVSTAT_* bits set by kernels whose bounded waits gave up.
+ * This call synchronises the device.  0 means no kernel gave up.
+ */
+int mla_device_status(unsigned int* status, int reset);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one CTA that waits on
+ * an mbarrier nothing will ever arrive on, with a time limit of
+ * `timeout_us` microseconds (1..10,000,000).  The kernel gives up, sets
+ * MLA_DEVSTAT_WAIT_TIMEOUT_TEST in the status word and returns normally.
+ */
+int mla_debug_wait_timeout(int timeout_us, mla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,217 @@
+"""ctypes binding of libmla.so (argument marshalling only).
+
+Every function here checks tensor dtypes/shapes/devices, allocates outputs
+with PyTorch when the caller passes none, and calls the C entry point of
+the same name on the current CUDA stream.  All computation happens in the
+library's CUDA kernels; if the library is missing or fails to load, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libmla.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_CUDA = 3
+DEVSTAT_WAIT_TIMEOUT_LOAD = 0x1
+DEVSTAT_WAIT_TIMEOUT_MMA = 0x2
+DEVSTAT_WAIT_TIMEOUT_SOFTMAX = 0x4
+DEVSTAT_WAIT_TIMEOUT_TEST = 0x100
+
+QK_DIM, V_DIM = 192, 128
+LATENT_DIM, LATENT_V_DIM = 576, 512
+
+# name -> (restype, argtypes), mirroring include/mla.h
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "mla_status_string": (ctypes.c_char_p, [_I]),
+    "mla_version": (_I, []),
+    "mla_prefill_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I]),
+    "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "mla_sparse_prefill_fwd": (_I, [_P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I]),
+    "mla_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
+    "mla_debug_wait_timeout": (_I, [_I, _P]),
+}
+
+
+class MlaError(RuntimeError):
+    """A libmla call returned an error status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libmla.so (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmla.so not built ({LIB_PATH}); run "
+                               "`python -m mla_prefill_attention_causal_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().mla_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MLA_OK:
+        raise MlaError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                    max_seqlen_q: int, max_seqlen_k: int,
+                    softmax_scale: Optional[float] = None, causal: bool = True,
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    return_lse: bool = True):
+    """Dense varlen MLA prefill forward (``mla_prefill_fwd`` in ``mla.h``).
+
+    q ``[total_q, H, 192]``, k ``[total_k, H, 192]``, v ``[total_k, H, 128]``
+    (bf16, contiguous, CUDA); cu_seqlens int32 ``[B+1]`` on the same device.
+    Returns ``(out [total_q, H, 128] bf16, lse [H, total_q] fp32 or None)``.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, num_heads, dq = q.shape
+    total_k = k.shape[0]
+    if dq != QK_DIM or k.shape[1:] != (num_heads, QK_DIM) or v.shape != (total_k, num_heads, V_DIM):
+        raise ValueError(f"MLA dims must be q/k [*, H, {QK_DIM}], v [*, H, {V_DIM}]; got "
+                         f"{tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    batch = cu_seqlens_q.numel() - 1
+    if batch < 1 or cu_seqlens_k.numel() != batch + 1:
+        raise ValueError("cu_seqlens_q/k must both have batch+1 >= 2 entries")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(QK_DIM)
+    if out is None:
+        out = torch.empty((total_q, num_heads, V_DIM), dtype=torch.bfloat16, device=q.device)
+    else:
+        _need(out, "out", torch.bfloat16, 3)
+        if out.shape != (total_q, num_heads, V_DIM):
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((num_heads, total_q), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+        if lse.shape != (num_heads, total_q):
+            raise ValueError("lse must be [num_heads, total_q]")
+    st = load().mla_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                int(max_seqlen_q), int(max_seqlen_k), float(softmax_scale),
+                                1 if causal else 0, _ptr(out), _ptr(lse), _stream(),
+                                batch, num_heads, total_q, total_k)
+    _check("mla_prefill_fwd", st)
+    return out, lse
+
+
+def mla_attn_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor,
+                   lse_b: torch.Tensor, out: Optional[torch.Tensor] = None,
+                   lse_out: Optional[torch.Tensor] = None, return_lse: bool = True):
+    """LSE merge of two partial results (``mla_attn_merge`` in ``mla.h``).
+
+    o ``[T, H, D]`` bf16, lse ``[H, T]`` fp32.  ``out`` may be ``o_a`` or
+    ``o_b``; ``lse_out`` must be a separate buffer.
+    """
+    for t, n in ((o_a, "o_a"), (o_b, "o_b")):
+        _need(t, n, torch.bfloat16, 3)
+    for t, n in ((lse_a, "lse_a"), (lse_b, "lse_b")):
+        _need(t, n, torch.float32, 2)
+    T, H, D = o_a.shape
+    if o_b.shape != o_a.shape or lse_a.shape != (H, T) or lse_b.shape != (H, T):
+        raise ValueError("shape mismatch between partial results")
+    if out is None:
+        out = torch.empty_like(o_a)
+    else:
+        _need(out, "out", torch.bfloat16, 3)
+    if lse_out is None and return_lse:
+        lse_out = torch.empty_like(lse_a)
+    st = load().mla_attn_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
+                               _ptr(lse_out), T, H, D, _stream())
+    _check("mla_attn_merge", st)
+    return out, lse_out
+
+
+def mla_sparse_prefill_fwd(q: torch.Tensor, kv_latent: torch.Tensor, indices: torch.Tensor,
+                           softmax_scale: Optional[float] = None,
+                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                           return_lse: bool = True):
+    """Absorbed top-k sparse MLA prefill (``mla_sparse_prefill_fwd``).
+
+    q ``[T, H, 576]`` bf16, kv_latent ``[N, 576]`` bf16, indices ``[T, topk]``
+    int32 (values outside ``[0, N)`` are padding).  Returns
+    ``(out [T, H, 512] bf16, lse [H, T] fp32 or None)``.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kv_latent, "kv_latent", torch.bfloat16, 2)
+    _need(indices, "indices", torch.int32, 2)
+    T, H, D = q.shape
+    N = kv_latent.shape[0]
+    if D != LATENT_DIM or kv_latent.shape[1] != LATENT_DIM or indices.shape[0] != T:
+        raise ValueError("sparse shapes must be q [T, H, 576], kv [N, 576], indices [T, topk]")
+    topk = indices.shape[1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(LATENT_DIM)
+    if out is None:
+        out = torch.empty((T, H, LATENT_V_DIM), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    st = load().mla_sparse_prefill_fwd(_ptr(q), _ptr(kv_latent), _ptr(indices), topk,
+                                       float(softmax_scale), _ptr(out), _ptr(lse), _stream(),
+                                       T, H, N)
+    _check("mla_sparse_prefill_fwd", st)
+    return out, lse
+
+
+def mla_device_status(reset: bool = True) -> int:
+    """OR of the device status bits set by kernels whose waits gave up."""
+    v = ctypes.c_uint(0)
+    _check("mla_device_status", load().mla_device_status(ctypes.byref(v), 1 if reset else 0))
+    return int(v.value)
+
+
+def mla_debug_wait_timeout(timeout_us: int) -> None:
+    """Launch the bounded-wait probe kernel (see ``mla.h``)."""
+    _check("mla_debug_wait_timeout", load().mla_debug_wait_timeout(int(timeout_us), _stream()))

@@ -1,0 +1,253 @@
+// libmla: the C-ABI entry points declared in include/mla.h.
+//
+// Host side only: argument validation, TMA tensor-map encoding (through the
+// driver entry point, so the library needs no -lcuda), launch configuration
+// and status mapping.  Every step of the computation runs in the kernels
+// included below; there is no host fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "dense_fwd.cuh"
+#include "merge.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // 4 s per barrier wait
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t t = []() -> uint64_t {
+    const char* e = std::getenv("MLA_WAIT_TIMEOUT_MS");
+    if (e != nullptr) {
+      const long long ms = std::atoll(e);
+      if (ms > 0 && ms < 600000) return static_cast<uint64_t>(ms) * 1000000ull;
+    }
+    return kDefaultTimeoutNs;
+  }();
+  return t;
+}
+
+// Per-device one-time state: architecture check and kernel attributes.
+struct DeviceState {
+  int checked = 0;  // 0 unknown, 1 ok, -1 unsupported
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int prepare_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  if (g_dev[dev].checked == 1) return MLA_OK;
+  if (g_dev[dev].checked == -1) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (g_dev[dev].checked != 0) return g_dev[dev].checked == 1 ? MLA_OK : MLA_ERR_UNSUPPORTED;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (major != 10 || minor != 0) {
+    g_dev[dev].checked = -1;
+    return MLA_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(mla::dense::dense_fwd_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           mla::dense::kSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (encode_fn() == nullptr) return MLA_ERR_CUDA;
+  g_dev[dev].checked = 1;
+  return MLA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a
+// 64-column x 128-row box and the 128-byte swizzle.  Rows past `rows` read
+// as zero.
+int encode_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                                 dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+__global__ void wait_timeout_probe(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mla::mbar_init(mla::smem_u32(&bar), 1);
+    abort_flag = 0;
+    mla::fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must give up after limit_ns.
+  mla::mbar_wait(mla::smem_u32(&bar), 0, &abort_flag, MLA_DEVSTAT_WAIT_TIMEOUT_TEST, limit_ns);
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK:
+      return "MLA_OK";
+    case MLA_ERR_INVALID_ARG:
+      return "MLA_ERR_INVALID_ARG: invalid argument (null/misaligned pointer or bad size)";
+    case MLA_ERR_UNSUPPORTED:
+      return "MLA_ERR_UNSUPPORTED: needs an sm_100 (B200) GPU and the supported shapes";
+    case MLA_ERR_CUDA:
+      return "MLA_ERR_CUDA: a CUDA call or kernel launch failed";
+    default:
+      return "unknown mla_status";
+  }
+}
+
+int mla_version(void) { return 100; }
+
+int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+                    float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
+                    int batch, int num_heads, int total_q, int total_k) {
+  using namespace mla::dense;
+  if (q == nullptr || k == nullptr || v == nullptr || cu_seqlens_q == nullptr ||
+      cu_seqlens_k == nullptr || out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || (lse && !aligned(lse, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || num_heads < 1 || num_heads > 65535 || total_q < 0 ||
+      total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || (causal != 0 && causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  int st = prepare_device(&dev);
+  if (st != MLA_OK) return st;
+  if (total_q == 0 || max_seqlen_q == 0) return MLA_OK;  // nothing to compute
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t kv_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  if ((st = encode_rows(&tq, q, static_cast<uint64_t>(num_heads) * kDqk, total_q)) != MLA_OK ||
+      (st = encode_rows(&tk, k, static_cast<uint64_t>(num_heads) * kDqk, kv_rows)) != MLA_OK ||
+      (st = encode_rows(&tv, v, static_cast<uint64_t>(num_heads) * kDv, kv_rows)) != MLA_OK)
+    return st;
+
+  Params p;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_heads = num_heads;
+  p.total_q = total_q;
+  p.causal = causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+  p.timeout_ns = wait_timeout_ns();
+  const dim3 grid((max_seqlen_q + kCtaRows - 1) / kCtaRows, num_heads, batch);
+  dense_fwd_kernel<<<grid, kThreads, kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk,
+                                                                                       tv, p);
+  return launch_status();
+}
+
+int mla_attn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                   void* out, float* lse_out, int num_tokens, int num_heads, int head_dim,
+                   mla_stream_t stream) {
+  if (o_a == nullptr || o_b == nullptr || lse_a == nullptr || lse_b == nullptr || out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(o_a, 16) || !aligned(o_b, 16) || !aligned(out, 16) || !aligned(lse_a, 4) ||
+      !aligned(lse_b, 4) || (lse_out && !aligned(lse_out, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (lse_out != nullptr && (lse_out == lse_a || lse_out == lse_b)) return MLA_ERR_INVALID_ARG;
+  if (num_tokens < 0 || num_heads < 1 || head_dim < 8 || head_dim % 8 != 0)
+    return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  int st = prepare_device(&dev);
+  if (st != MLA_OK) return st;
+  if (num_tokens == 0) return MLA_OK;
+  const long long rows = static_cast<long long>(num_tokens) * num_heads;
+  const int vpr = head_dim / 8;
+  const long long vecs = rows * vpr;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (vecs + mla::merge::kThreads - 1) / mla::merge::kThreads;
+  const long long cap = static_cast<long long>(sms) * 8;  // 8 resident CTAs of 256 per SM
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  mla::merge::merge_kernel<<<blocks, mla::merge::kThreads, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
+      static_cast<uint4*>(out), lse_out, rows, num_heads, num_tokens, vpr);
+  return launch_status();
+}
+
+int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* indices, int topk,
+                           float softmax_scale, void* out, float* lse, mla_stream_t stream,
+                           int num_tokens, int num_heads, int num_kv_rows) {
+  if (q == nullptr || kv_latent == nullptr || indices == nullptr || out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv_latent, 16) || !aligned(out, 16) || !aligned(indices, 4) ||
+      (lse && !aligned(lse, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (topk < 1 || num_tokens < 0 || num_heads < 1 || num_heads > 128 || num_kv_rows < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  (void)stream;
+  return MLA_ERR_UNSUPPORTED;
+}
+
+int mla_device_status(unsigned int* status, int reset) {
+  if (status == nullptr) return MLA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(status, mla::g_mla_status, sizeof(unsigned int)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (reset) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(mla::g_mla_status, &zero, sizeof(zero)) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+int mla_debug_wait_timeout(int timeout_us, mla_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 10000000) return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  int st = prepare_device(&dev);
+  if (st != MLA_OK) return st;
+  wait_timeout_probe<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  return launch_status();
+}
+
+}  // extern "C"

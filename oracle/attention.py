@@ -98,49 +98,47 @@ def dense_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale: float,
       cu_seqlens_q / cu_seqlens_k: ``[B+1]`` prefix sums.
       softmax_scale: the scale applied to every ``q . k`` product.
       causal: bottom-right causal mask when true.
-      rows: optional iterable of global query rows to evaluate (all if None).
+      rows: optional sequence of global query rows to evaluate.
 
-    Returns ``(out, lse)``: float64 ``out [total_q, H, Dv]`` and
-    ``lse [H, total_q]``.  Rows that were not evaluated hold NaN.
+    Returns ``(out, lse)`` in float64: ``out [R, H, Dv]`` and ``lse [H, R]``
+    where R runs over all query rows in order (``rows=None``) or over the
+    given rows in the given order.  bf16 inputs are widened one
+    (sequence, head) slice at a time.
     """
-    q = _as_f64(q)
-    k = _as_f64(k)
-    v = _as_f64(v)
     cu_q = np.asarray(cu_seqlens_q, dtype=np.int64)
     cu_k = np.asarray(cu_seqlens_k, dtype=np.int64)
     total_q, num_heads, _ = q.shape
     dv = v.shape[2]
-    out = np.full((total_q, num_heads, dv), np.nan)
-    lse = np.full((num_heads, total_q), np.nan)
-    wanted = None if rows is None else np.zeros(total_q, dtype=bool)
-    if wanted is not None:
-        wanted[np.asarray(list(rows), dtype=np.int64)] = True
+    sel_rows = np.arange(total_q) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    out = np.zeros((sel_rows.size, num_heads, dv))
+    lse = np.zeros((num_heads, sel_rows.size))
+    seq_of = np.searchsorted(cu_q, sel_rows, side="right") - 1
     scale = float(softmax_scale)
 
-    for b in range(len(cu_q) - 1):
+    for b in np.unique(seq_of):
         q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
         k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
         lq, lk = q1 - q0, k1 - k0
-        local = np.arange(lq) if wanted is None else np.nonzero(wanted[q0:q1])[0]
-        if local.size == 0:
-            continue
+        pos = np.nonzero(seq_of == b)[0]          # positions in the output
+        local = sel_rows[pos] - q0                # rows within the sequence
         counts_all = np.array([visible_key_count(int(i), lq, lk, causal)
                                for i in local], dtype=np.int64)
         for h in range(num_heads):
-            kb = k[k0:k1, h, :]
-            vb = v[k0:k1, h, :]
+            kb = _as_f64(k[k0:k1, h, :])
+            vb = _as_f64(v[k0:k1, h, :])
             for g in range(0, local.size, row_group):
                 sel = local[g:g + row_group]
+                dst = pos[g:g + row_group]
                 counts = counts_all[g:g + row_group]
-                scores = scale * (q[q0 + sel, h, :] @ kb.T)
+                scores = scale * (_as_f64(q[q0 + sel, h, :]) @ kb.T)
                 e, row_max, z = _softmax_rows(scores, counts)
                 has = z > 0
                 o = np.zeros((sel.size, dv))
                 o[has] = (e[has] @ vb) / z[has, None]
-                out[q0 + sel, h, :] = o
+                out[dst, h, :] = o
                 with np.errstate(divide="ignore"):
-                    lse[h, q0 + sel] = np.where(has, row_max + np.log(np.where(has, z, 1.0)),
-                                                -np.inf)
+                    lse[h, dst] = np.where(has, row_max + np.log(np.where(has, z, 1.0)),
+                                           -np.inf)
     return out, lse
 
 
@@ -184,32 +182,31 @@ def sparse_prefill(q, kv, indices, softmax_scale: float, v_dim: int = 512,
     kv_r[:v_dim]``; ``lse[h, t]`` is the natural log-sum-exp of the scores.
 
     Shapes: ``q [T, H, Dl]``, ``kv [N, Dl]``, ``indices [T, K]`` int.
-    Returns ``out [T, H, v_dim]`` and ``lse [H, T]`` (float64); tokens not
-    listed in ``tokens`` hold NaN.
+    Returns float64 ``out [R, H, v_dim]`` and ``lse [H, R]`` with R running
+    over all tokens (``tokens=None``) or over the given tokens in order.
     """
-    q = _as_f64(q)
     kv = _as_f64(kv)
     idx = np.asarray(indices, dtype=np.int64)
     num_tokens, num_heads, _ = q.shape
     num_rows = kv.shape[0]
-    out = np.full((num_tokens, num_heads, v_dim), np.nan)
-    lse = np.full((num_heads, num_tokens), np.nan)
+    todo = np.arange(num_tokens) if tokens is None else np.asarray(list(tokens), dtype=np.int64)
+    out = np.zeros((todo.size, num_heads, v_dim))
+    lse = np.zeros((num_heads, todo.size))
     scale = float(softmax_scale)
-    todo = range(num_tokens) if tokens is None else tokens
-    for t in todo:
+    for pos, t in enumerate(todo):
         t = int(t)
         row_ids = idx[t]
         row_ids = row_ids[(row_ids >= 0) & (row_ids < num_rows)]
         if row_ids.size == 0:
-            out[t] = 0.0
-            lse[:, t] = -np.inf
+            out[pos] = 0.0
+            lse[:, pos] = -np.inf
             continue
-        sel = kv[row_ids]                       # [n, Dl]
-        scores = scale * (q[t] @ sel.T)         # [H, n]
+        sel = kv[row_ids]                             # [n, Dl]
+        scores = scale * (_as_f64(q[t]) @ sel.T)      # [H, n]
         counts = np.full(num_heads, row_ids.size, dtype=np.int64)
         e, row_max, z = _softmax_rows(scores, counts)
-        out[t] = (e @ sel[:, :v_dim]) / z[:, None]
-        lse[:, t] = row_max + np.log(z)
+        out[pos] = (e @ sel[:, :v_dim]) / z[:, None]
+        lse[:, pos] = row_max + np.log(z)
     return out, lse
 
 

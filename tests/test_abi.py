@@ -1,0 +1,91 @@
+"""The C-ABI library: it loads, exports every declared symbol, and rejects
+bad arguments on the host before touching a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_prefill_attention_causal_b200 as mla
+from mla_prefill_attention_causal_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(mla_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("mla_prefill_fwd", "mla_attn_merge", "mla_sparse_prefill_fwd",
+                 "mla_status_string", "mla_device_status"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version():
+    assert mla.status_string(0) == "MLA_OK"
+    assert "INVALID_ARG" in mla.status_string(1)
+    assert "UNSUPPORTED" in mla.status_string(2)
+    assert mla.load().mla_version() >= 100
+
+
+def _call_dense(**over):
+    a = dict(q=16, k=16, v=16, cq=16, ck=16, mq=4, mk=4, scale=0.1, causal=1, out=16, lse=None,
+             stream=None, batch=1, H=1, tq=4, tk=4)
+    a.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return mla.load().mla_prefill_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["cq"]), P(a["ck"]),
+                                      a["mq"], a["mk"], a["scale"], a["causal"], P(a["out"]),
+                                      P(a["lse"]), None, a["batch"], a["H"], a["tq"], a["tk"])
+
+
+@pytest.mark.parametrize("over", [dict(q=None), dict(out=None), dict(cq=None), dict(q=24),
+                                  dict(out=8), dict(cq=2), dict(batch=0), dict(H=0),
+                                  dict(tq=-1), dict(causal=2), dict(scale=0.0),
+                                  dict(scale=float("nan")), dict(scale=-1.0), dict(lse=2)])
+def test_dense_rejects_bad_arguments(over):
+    assert _call_dense(**over) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_merge_rejects_bad_arguments():
+    f = mla.load().mla_attn_merge
+    P = ctypes.c_void_p
+    ok = dict(oa=16, la=16, ob=16, lb=16, out=16, lo=32, T=4, H=2, D=128)
+
+    def call(**over):
+        a = dict(ok)
+        a.update(over)
+        p = lambda x: None if x is None else P(x)
+        return f(p(a["oa"]), p(a["la"]), p(a["ob"]), p(a["lb"]), p(a["out"]), p(a["lo"]),
+                 a["T"], a["H"], a["D"], None)
+    assert call(oa=None) == _lib.MLA_ERR_INVALID_ARG
+    assert call(D=12) == _lib.MLA_ERR_INVALID_ARG
+    assert call(lo=16) == _lib.MLA_ERR_INVALID_ARG      # lse_out aliases lse_a
+    assert call(out=40) == _lib.MLA_ERR_INVALID_ARG     # misaligned
+    assert call(T=-1) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_sparse_rejects_bad_arguments():
+    f = mla.load().mla_sparse_prefill_fwd
+    P = ctypes.c_void_p
+    assert f(None, P(16), P(16), 8, 0.1, P(16), None, None, 4, 128, 10) == _lib.MLA_ERR_INVALID_ARG
+    assert f(P(16), P(16), P(16), 0, 0.1, P(16), None, None, 4, 128, 10) == _lib.MLA_ERR_INVALID_ARG
+    assert f(P(16), P(16), P(16), 8, 0.1, P(16), None, None, 4, 129, 10) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libmla.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        _lib.load()

@@ -1,0 +1,138 @@
+"""Parity of the CUDA dense MLA prefill (through the C ABI) with the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import mla_synth as syn
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+from gpu_util import (assert_lse_close, assert_out_close, check_dense, dev_bf16, dev_i32,  # noqa: E402
+                      run_dense, sample_rows, to_f64)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean(cuda_ok):
+    import mla_prefill_attention_causal_b200 as mla
+    mla.mla_device_status(reset=True)
+    yield
+    assert mla.mla_device_status(reset=True) == 0, "a kernel wait gave up"
+
+
+def test_tiny_config_full():
+    """2 ragged sequences (64, 100), 4 heads, causal: every row and head."""
+    check_dense(syn.tiny_config())
+
+
+@pytest.mark.parametrize("lens", [[1, 127, 128, 129], [255, 256, 257, 300], [511, 513, 1]])
+def test_tile_edge_lengths_causal(lens):
+    check_dense(syn.dense_case(lens, lens, 3, seed=sum(lens)))
+
+
+def test_noncausal_ragged_lq_ne_lk():
+    check_dense(syn.dense_case([1, 129, 200, 64], [128, 512, 77, 1], 2, seed=11, causal=False))
+
+
+def test_causal_bottom_right_lq_lt_lk():
+    check_dense(syn.dense_case([100, 300, 1], [400, 333, 700], 2, seed=12, causal=True))
+
+
+def test_causal_lq_gt_lk_rows_without_keys():
+    """Bottom-right causal with Lq > Lk: the first Lq-Lk rows see no key."""
+    case = syn.dense_case([200, 150], [50, 150], 2, seed=13, causal=True)
+    out, lse = run_dense(case)
+    check_dense(case)
+    o = to_f64(out)
+    assert np.all(o[:150] == 0) and np.all(np.isneginf(lse[:, :150].cpu().numpy()))
+
+
+def test_empty_key_sequence():
+    case = syn.dense_case([40, 70], [0, 90], 2, seed=14, causal=False)
+    out, lse = run_dense(case)
+    check_dense(case)
+    assert np.all(to_f64(out)[:40] == 0)
+
+
+@pytest.mark.parametrize("max_q,max_k", [(1, 128), (129, 512), (1, 4096), (129, 4096)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_warmup_probe_shapes(max_q, max_k, causal):
+    """The (max_seqlen_q, max_seqlen_k) shape probes of vLLM's FA4 MLA warmup."""
+    case = syn.dense_case([max_q], [max_k], 2, seed=max_q + max_k, causal=causal)
+    check_dense(case)
+
+
+def test_lse_optional_and_out_identical():
+    case = syn.dense_case([300, 77], [300, 77], 2, seed=15)
+    o1, l1 = run_dense(case, want_lse=True)
+    o2, l2 = run_dense(case, want_lse=False)
+    assert l2 is None
+    assert torch.equal(o1, o2)
+
+
+def test_bitwise_deterministic():
+    case = syn.dense_case([700, 1300, 257], [700, 1300, 257], 8, seed=16)
+    o1, l1 = run_dense(case)
+    o2, l2 = run_dense(case)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_batch_invariant():
+    """A sequence gives identical bits alone and inside a batch."""
+    lens = [300, 1000, 129]
+    case = syn.dense_case(lens, lens, 4, seed=17)
+    o_all, l_all = run_dense(case)
+    s0, s1 = int(case["cu_q"][1]), int(case["cu_q"][2])
+    alone = dict(case)
+    alone.update(q=case["q"][s0:s1], k=case["k"][s0:s1], v=case["v"][s0:s1],
+                 cu_q=syn.cu_seqlens([lens[1]]), cu_k=syn.cu_seqlens([lens[1]]),
+                 max_q=lens[1], max_k=lens[1])
+    o1, l1 = run_dense(alone)
+    assert torch.equal(o1, o_all[s0:s1])
+    assert torch.equal(l1, l_all[:, s0:s1])
+
+
+def test_many_heads_small():
+    lens = [383, 129]
+    check_dense(syn.dense_case(lens, lens, 128, seed=18))
+
+
+def test_varlen16k_config_sampled():
+    """8 sequences, lengths U[512,4096], 128 heads: sampled rows, all heads."""
+    case = syn.varlen16k_config()
+    check_dense(case, rows=sample_rows(case["lens_q"], seed=2))
+
+
+def test_long32k_config_sampled():
+    """One 32768-token sequence, 128 heads: 300+ sampled rows, all heads."""
+    case = syn.long32k_config()
+    rows = sample_rows(case["lens_q"], seed=3, per_seq=300)
+    rows += [r for r in range(4095, 32768, 4096)]
+    check_dense(case, rows=sorted(set(rows)))
+
+
+def test_chunked_prefill_with_context_merge():
+    """Prefix pass (unmasked, LSE) + self pass (causal) + merge equals one
+    bottom-right causal pass over [prefix, chunk] (sampled rows)."""
+    import mla_prefill_attention_causal_b200 as mla
+    d = syn.chunked_config()
+    q = dev_bf16(d["q"])
+    kp, vp = dev_bf16(d["k_prefix"]), dev_bf16(d["v_prefix"])
+    ks, vs = dev_bf16(d["k_self"]), dev_bf16(d["v_self"])
+    cq, cp = dev_i32(d["cu_q"]), dev_i32(d["cu_prefix"])
+    o1, l1 = mla.mla_prefill_fwd(q, kp, vp, cq, cp, d["chunk"], d["prefix"], d["scale"], causal=False)
+    o2, l2 = mla.mla_prefill_fwd(q, ks, vs, cq, cq, d["chunk"], d["chunk"], d["scale"], causal=True)
+    om, lm = mla.mla_attn_merge(o1, l1, o2, l2)
+    torch.cuda.synchronize()
+    B, C, P, H = d["batch"], d["chunk"], d["prefix"], d["num_heads"]
+    rows = sample_rows([C] * B, seed=4, per_seq=12)
+    # oracle: one causal call over the concatenated keys of each sequence
+    k_cat = np.concatenate([np.concatenate([d["k_prefix"][b * P:(b + 1) * P],
+                                            d["k_self"][b * C:(b + 1) * C]]) for b in range(B)])
+    v_cat = np.concatenate([np.concatenate([d["v_prefix"][b * P:(b + 1) * P],
+                                            d["v_self"][b * C:(b + 1) * C]]) for b in range(B)])
+    ref_o, ref_l = oracle.dense_prefill(d["q"], k_cat, v_cat, d["cu_q"],
+                                        syn.cu_seqlens([P + C] * B), d["scale"], True, rows=rows)
+    idx = torch.as_tensor(rows, device=om.device)
+    assert_out_close(to_f64(om.index_select(0, idx)), ref_o, "merged out")
+    assert_lse_close(lm.index_select(1, idx).cpu().numpy().astype(np.float64), ref_l, "merged lse")

@@ -58,6 +58,7 @@ typedef enum {
 #define MLA_DEVSTAT_WAIT_TIMEOUT_LOAD 0x1u    /* load warp gave up waiting    */
 #define MLA_DEVSTAT_WAIT_TIMEOUT_MMA 0x2u     /* MMA warp gave up waiting     */
 #define MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX 0x4u /* softmax warps gave up waiting */
+#define MLA_DEVSTAT_PLAN_OVERFLOW 0x10u       /* cu_seqlens_q[batch] > total_q */
 #define MLA_DEVSTAT_WAIT_TIMEOUT_TEST 0x100u  /* mla_debug_wait_timeout probe  */
 
 /* Human-readable text for an mla_status value (static storage). */
@@ -65,6 +66,14 @@ const char* mla_status_string(int status);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int mla_version(void);
+
+/*
+ * Bytes of device workspace mla_prefill_fwd needs for a call with these
+ * sizes: a small header plus one 8-byte entry per (sequence, 256-row query
+ * block), at most ceil(total_q / 256) + batch of them.  Returns 0 for
+ * invalid sizes.
+ */
+size_t mla_prefill_workspace_size(int batch, int total_q);
 
 /*
  * Dense varlen MLA prefill forward.
@@ -78,6 +87,10 @@ int mla_version(void);
  * backend's run_prefill_new_tokens; causal == 0 with a separate key set is
  * its run_prefill_context_chunk).
  *
+ * Two kernels are enqueued: a one-CTA planner that orders the work (longest
+ * first) into `workspace`, and a persistent attention kernel (one CTA per
+ * SM) that consumes it.
+ *
  * Arguments:
  *   q            bf16 [total_q, num_heads, 192], contiguous, 16-B aligned.
  *   k            bf16 [total_k, num_heads, 192], contiguous, 16-B aligned.
@@ -86,21 +99,27 @@ int mla_version(void);
  *                cu[batch] = total_q.  Sequence b owns query rows
  *                [cu_q[b], cu_q[b+1]).
  *   cu_seqlens_k int32 [batch+1] on the device, same rules for keys.
- *   max_seqlen_q upper bound on cu_q[b+1] - cu_q[b] (rows past it are not
- *                computed); max_seqlen_k likewise for keys (informational).
+ *   max_seqlen_q, max_seqlen_k  informational upper bounds (>= 0); the
+ *                kernels take the lengths from cu_seqlens.
  *   softmax_scale finite, > 0; multiplies q.k (1/sqrt(192) for MLA).
  *   causal       0 or 1.
  *   out          bf16 [total_q, num_heads, 128], 16-B aligned; fully written.
  *   lse          float32 [num_heads, total_q] or NULL (not returned).
  *   stream       stream to enqueue on.
  *   batch, num_heads, total_q, total_k: sizes (total_* >= 0, batch >= 1,
- *                1 <= num_heads <= 65535, batch <= 65535).
+ *                1 <= num_heads <= 65535).
+ *   workspace    device memory of at least mla_prefill_workspace_size(batch,
+ *                total_q) bytes, 16-B aligned, owned by the caller; its
+ *                contents need no initialisation.  Calls that may run at the
+ *                same time (different streams) need separate workspaces.
+ *   workspace_bytes  its size (MLA_ERR_INVALID_ARG if too small).
  * Returns MLA_OK or an error; on error nothing was launched.
  */
 int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
                     const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
                     float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
-                    int batch, int num_heads, int total_q, int total_k);
+                    int batch, int num_heads, int total_q, int total_k, void* workspace,
+                    size_t workspace_bytes);
 
 /*
  * Merge two partial attention results over disjoint key sets A and B into

@@ -13,5 +13,6 @@ from ._lib import (  # noqa: F401
     mla_device_status,
     mla_prefill_fwd,
     mla_sparse_prefill_fwd,
+    prefill_workspace_size,
     status_string,
 )

@@ -35,7 +35,9 @@ _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "mla_status_string": (ctypes.c_char_p, [_I]),
     "mla_version": (_I, []),
-    "mla_prefill_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I]),
+    "mla_prefill_workspace_size": (_S, [_I, _I]),
+    "mla_prefill_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P,
+                             _S]),
     "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "mla_sparse_prefill_fwd": (_I, [_P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I]),
     "mla_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
@@ -105,11 +107,13 @@ def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     max_seqlen_q: int, max_seqlen_k: int,
                     softmax_scale: Optional[float] = None, causal: bool = True,
                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                    return_lse: bool = True):
+                    return_lse: bool = True, workspace: Optional[torch.Tensor] = None):
     """Dense varlen MLA prefill forward (``mla_prefill_fwd`` in ``mla.h``).
 
     q ``[total_q, H, 192]``, k ``[total_k, H, 192]``, v ``[total_k, H, 128]``
     (bf16, contiguous, CUDA); cu_seqlens int32 ``[B+1]`` on the same device.
+    ``workspace`` (uint8, >= ``prefill_workspace_size(B, total_q)`` bytes) is
+    allocated from PyTorch's stream-ordered allocator when not given.
     Returns ``(out [total_q, H, 128] bf16, lse [H, total_q] fp32 or None)``.
     """
     _need(q, "q", torch.bfloat16, 3)
@@ -139,12 +143,23 @@ def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         _need(lse, "lse", torch.float32, 2)
         if lse.shape != (num_heads, total_q):
             raise ValueError("lse must be [num_heads, total_q]")
+    ws_bytes = prefill_workspace_size(batch, total_q)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < ws_bytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of >= {ws_bytes} bytes")
     st = load().mla_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
                                 int(max_seqlen_q), int(max_seqlen_k), float(softmax_scale),
                                 1 if causal else 0, _ptr(out), _ptr(lse), _stream(),
-                                batch, num_heads, total_q, total_k)
+                                batch, num_heads, total_q, total_k, _ptr(workspace),
+                                workspace.numel() * workspace.element_size())
     _check("mla_prefill_fwd", st)
     return out, lse
+
+
+def prefill_workspace_size(batch: int, total_q: int) -> int:
+    """Workspace bytes ``mla_prefill_fwd`` needs (``mla_prefill_workspace_size``)."""
+    return int(load().mla_prefill_workspace_size(int(batch), int(total_q)))
 
 
 def mla_attn_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor,

@@ -7,22 +7,39 @@
 // dims of vLLM's flash_attn.py MLA prefill backend (qk 128 nope + 64 rope =
 // 192, v 128, K/V expanded per head).
 //
-// One CTA owns one (sequence, 256-row query block, head) tile, split into
-// two 128-row sub-tiles that share every K/V block:
-//   warps 0-3  softmax for sub-tile 0 (thread = query row = TMEM lane)
-//   warps 4-7  softmax for sub-tile 1
-//   warp  8    TMA producer: Q once, then K/V chunks into an 8-slot ring
-//   warp  9    MMA issuer (one thread): S = Q K^T and O += P V (tcgen05)
-// Shared memory: Q 96 KB (2 sub-tiles x 3 chunks of 128 rows x 64 dims) and
-// a ring of 8 chunks of 16 KB; every chunk is a 128-row x 128-byte tile with
-// the 128-byte swizzle that both TMA and the MMA descriptors use.  A K block
-// (128 keys x 192 dims) is 3 chunks, a V block (128 keys x 128 dims) 2.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
-// P_i (bf16, 64 columns) overwrites the first half of S_i once S_i is read.
+// The kernel runs on CTA pairs (clusters of 2 on one TPC) and issues M=256
+// tcgen05 MMAs with cta_group::2: each CTA keeps its own 128 query rows of
+// an MMA in shared memory and TMEM, while each K/V block is split between
+// the two CTAs (CTA r holds keys [64r, 64r+64) of every K block and value
+// dims [64r, 64r+64) of every V block).  Compared with one CTA per MMA this
+// halves each SM's K/V traffic and the shared-memory operand bytes per MMA.
+//
+// Work unit ("tile"): (sequence, 512-row query block, head) = two M=256
+// sub-tiles that share every K/V block.  A planner kernel sorts the
+// (sequence, query block) entries by their number of visible KV blocks,
+// longest first, into the caller's workspace; the persistent clusters walk
+// that list head-major in a static snake order (cluster c takes tile
+// k*C + c on even rounds and k*C + C-1-c on odd ones), so both CTAs of a
+// pair derive the same tile sequence without talking, clusters running at
+// the same time share K/V in L2, and the short tiles come last.
+//
+// Roles inside each CTA (320 threads):
+//   warps 0-3  softmax + epilogue, sub-tile 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax + epilogue, sub-tile 1
+//   warp  8    producer: TMA loads of this CTA's Q rows and K/V halves, whose
+//              completion is counted on the leader CTA's barriers
+//   warp  9    (leader CTA only) MMA issuer: S = Q K^T, O += P V
+// Shared memory per CTA: Q 96 KB (2 sub-tiles x 3 chunks of 128 rows x 64
+// dims) and a ring of 16 units of 8 KB (64 rows x 64 dims), all with the
+// 128-byte swizzle used by TMA and the MMA descriptors; one KV block takes
+// 5 units per CTA (3 for its K half, 2 for its V half).
+// TMEM per CTA (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1
+// [384,512); P_i (bf16, 64 columns) overwrites the first half of S_i.
 //
 // MMA issue order per KV block n (so one sub-tile's softmax overlaps the
-// other's MMAs): PV0(n), S0(n+1), PV1(n), S1(n+1).  Masking is applied only
-// to blocks that are not fully visible (the diagonal and the ragged end).
+// other's MMAs): PV0(n), S0(n+1), PV1(n), S1(n+1), where block n+1 may be
+// the first block of the next tile.  Masking is applied only to blocks that
+// are not fully visible (the diagonal and the ragged end).
 #pragma once
 #include <cuda_bf16.h>
 
@@ -31,29 +48,52 @@
 namespace mla {
 namespace dense {
 
-constexpr int kSubRows = 128;                        // MMA M (rows per sub-tile)
-constexpr int kCtaRows = 256;                        // query rows per CTA
-constexpr int kBlockKeys = 128;                      // keys per KV block
+constexpr int kCtaRows = 128;                        // rows of a sub-tile held by one CTA
+constexpr int kSubRows = 256;                        // MMA M (rows per sub-tile, both CTAs)
+constexpr int kTileRows = 512;                       // query rows per tile
+constexpr int kBlockKeys = 128;                      // keys per KV block (MMA N of S)
+constexpr int kHalfKeys = 64;                        // keys of a K block held by one CTA
 constexpr int kDqk = 192;
 constexpr int kDv = 128;
-constexpr int kChunkBytes = 128 * 128;               // 128 rows x 64 bf16
+constexpr int kHalfDv = 64;                          // value dims held by one CTA
+constexpr int kQChunkBytes = 128 * 128;              // 128 rows x 64 bf16
+constexpr int kUnitBytes = 64 * 128;                 // 64 rows x 64 bf16
 constexpr int kQkChunks = kDqk / 64;                 // 3
-constexpr int kVChunks = kDv / 64;                   // 2
-constexpr int kItemsPerBlock = kQkChunks + kVChunks; // 5 ring items per KV block
-constexpr int kRing = 8;
-constexpr int kQBytes = 2 * kQkChunks * kChunkBytes; // 96 KB
-constexpr int kRingBytes = kRing * kChunkBytes;      // 128 KB
+constexpr int kKUnits = kQkChunks;                   // K half: 64 keys x 192 dims
+constexpr int kVUnits = kBlockKeys / 64;             // V half: 128 keys x 64 dims
+constexpr int kItemsPerBlock = kKUnits + kVUnits;    // 5 ring units per KV block
+constexpr int kRing = 16;
+constexpr int kQSubBytes = kQkChunks * kQChunkBytes; // 48 KB
+constexpr int kQBytes = 2 * kQSubBytes;              // 96 KB
+constexpr int kRingBytes = kRing * kUnitBytes;       // 128 KB
 constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBins = 4096;                      // work histogram bins (clamped)
+
+// Workspace layout (caller-provided device memory, 16-byte aligned).
+struct WsHeader {
+  int num_entries;  // E: (sequence, 512-row block) entries
+  int num_tiles;    // E * num_heads
+  int pad[2];
+};
+constexpr size_t kWsHeaderBytes = 256;
+
+struct TileInfo {
+  int q_start, Lq, k_start, Lk;
+  int m0, h, valid, pad;
+};
 
 struct alignas(8) Bars {
-  uint64_t q_full;
-  uint64_t full[kRing];
-  uint64_t empty[kRing];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_full[2];
-  uint64_t drain;
+  uint64_t q_full[2];    // leader: Q bytes of both CTAs
+  uint64_t q_empty[2];   // both: last S MMA of the tile done
+  uint64_t full[kRing];  // leader: unit bytes of both CTAs
+  uint64_t empty[kRing]; // both: MMAs reading the unit done
+  uint64_t s_full[2];    // both
+  uint64_t p_full[2];    // leader: 8 softmax warps (both CTAs)
+  uint64_t o_full[2];    // both
+  uint64_t o_empty[2];   // leader: 8 softmax warps (both CTAs)
+  uint64_t drain;        // leader
   uint32_t tmem_base;
   int abort;
 };
@@ -65,6 +105,8 @@ struct Params {
   const int* cu_k;
   __nv_bfloat16* out;
   float* lse;
+  const WsHeader* ws;
+  const int2* entries;  // [E] {sequence, 512-row block index}, longest first
   int num_heads;
   int total_q;
   int causal;
@@ -72,17 +114,97 @@ struct Params {
   uint64_t timeout_ns;  // limit for every barrier wait
 };
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
-constexpr uint32_t kIdescPV128 = idesc_bf16_f32(128, 128, true);
-constexpr uint32_t kIdescPV64 = idesc_bf16_f32(128, 64, true);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(256, 128, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(256, 128, true);
 
-// Number of keys (a prefix [0, n)) that any row of the sub-tile starting at
-// row0 may see, and hence the KV blocks the sub-tile must visit.
-__device__ __forceinline__ int sub_tile_keys(int row0, int Lq, int Lk, int causal) {
+// Number of keys (a prefix [0, n)) that any row of the 256-row sub-tile
+// starting at row0 may see.
+__host__ __device__ __forceinline__ int sub_tile_keys(int row0, int Lq, int Lk, int causal) {
   if (row0 >= Lq) return 0;
   if (!causal) return Lk;
   const int last = min(row0 + kSubRows - 1, Lq - 1);
   return max(0, min(Lk, last + (Lk - Lq) + 1));
+}
+__host__ __device__ __forceinline__ int blocks_for(int keys) {
+  return (keys + kBlockKeys - 1) / kBlockKeys;
+}
+
+// ------------------------------------------------------------------ planner
+// One CTA: builds the (sequence, 512-row block) entry list sorted by the
+// number of KV blocks its rows visit (descending).
+__global__ void __launch_bounds__(kPlanThreads)
+    dense_plan_kernel(const int* cu_q, const int* cu_k, int batch, int causal, WsHeader* ws,
+                      int2* entries, int capacity, int num_heads) {
+  __shared__ int bins[kPlanBins];
+  __shared__ int s_total;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kPlanBins; i += blockDim.x) bins[i] = 0;
+  if (tid == 0) s_total = 0;
+  __syncthreads();
+  auto work_of = [&](int Lq, int Lk, int mb) -> int {
+    const int m0 = mb * kTileRows;
+    const int k0 = sub_tile_keys(m0, Lq, Lk, causal);
+    const int k1 = sub_tile_keys(m0 + kSubRows, Lq, Lk, causal);
+    return min(kPlanBins - 1, blocks_for(max(k0, k1)));
+  };
+  for (int b = tid; b < batch; b += blockDim.x) {
+    const int Lq = cu_q[b + 1] - cu_q[b];
+    const int Lk = cu_k[b + 1] - cu_k[b];
+    const int nmb = (Lq + kTileRows - 1) / kTileRows;
+    atomicAdd(&s_total, nmb);
+    for (int mb = 0; mb < nmb; ++mb) atomicAdd(&bins[work_of(Lq, Lk, mb)], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {  // exclusive prefix over bins in descending work order
+    int run = 0;
+    for (int w = kPlanBins - 1; w >= 0; --w) {
+      const int c = bins[w];
+      bins[w] = run;
+      run += c;
+    }
+    // More entries than the workspace holds means cu_seqlens_q does not end
+    // at total_q: report it and compute only what fits.
+    if (s_total > capacity) atomicOr(&g_mla_status, MLA_DEVSTAT_PLAN_OVERFLOW);
+    const int e = min(s_total, capacity);
+    ws->num_entries = e;
+    ws->num_tiles = e * num_heads;
+  }
+  __syncthreads();
+  for (int b = tid; b < batch; b += blockDim.x) {
+    const int Lq = cu_q[b + 1] - cu_q[b];
+    const int Lk = cu_k[b + 1] - cu_k[b];
+    const int nmb = (Lq + kTileRows - 1) / kTileRows;
+    for (int mb = nmb - 1; mb >= 0; --mb) {
+      const int pos = atomicAdd(&bins[work_of(Lq, Lk, mb)], 1);
+      if (pos < capacity) entries[pos] = make_int2(b, mb);
+    }
+  }
+}
+
+// Tile k of cluster c (static snake order over the sorted entry list).
+__device__ __forceinline__ TileInfo tile_at(const Params& p, int k, int cluster, int nclusters,
+                                            int num_tiles, int num_entries) {
+  const long long t = static_cast<long long>(k) * nclusters +
+                      ((k & 1) ? (nclusters - 1 - cluster) : cluster);
+  TileInfo ti;
+  ti.valid = t < num_tiles ? 1 : 0;
+  if (ti.valid) {
+    const int tt = static_cast<int>(t);
+    const int h = tt / num_entries;
+    const int2 e = p.entries[tt - h * num_entries];
+    ti.q_start = p.cu_q[e.x];
+    ti.Lq = p.cu_q[e.x + 1] - ti.q_start;
+    ti.k_start = p.cu_k[e.x];
+    ti.Lk = p.cu_k[e.x + 1] - ti.k_start;
+    ti.m0 = e.y * kTileRows;
+    ti.h = h;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ void tile_blocks(const TileInfo& t, int causal, int (&n)[2]) {
+  n[0] = t.valid ? blocks_for(sub_tile_keys(t.m0, t.Lq, t.Lk, causal)) : 0;
+  n[1] = t.valid ? blocks_for(sub_tile_keys(t.m0 + kSubRows, t.Lq, t.Lk, causal)) : 0;
 }
 
 __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
@@ -104,20 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int b = blockIdx.z;
-  const int h = blockIdx.y;
-  const int mb = gridDim.x - 1 - blockIdx.x;  // longest (causal) blocks first
-
-  const int q_start = p.cu_q[b];
-  const int Lq = p.cu_q[b + 1] - q_start;
-  const int k_start = p.cu_k[b];
-  const int Lk = p.cu_k[b + 1] - k_start;
-  const int m0 = mb * kCtaRows;
-  if (m0 >= Lq) return;  // uniform for the whole CTA
-  const int off = Lk - Lq;
-  const int nb0 = (sub_tile_keys(m0, Lq, Lk, p.causal) + kBlockKeys - 1) / kBlockKeys;
-  const int nb1 = (sub_tile_keys(m0 + kSubRows, Lq, Lk, p.causal) + kBlockKeys - 1) / kBlockKeys;
-  const int nblk = max(nb0, nb1);
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = static_cast<int>(blockIdx.x >> 1);
+  const int nclusters = static_cast<int>(gridDim.x >> 1);
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -125,299 +237,373 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sRing = sQ + kQBytes;
   Bars* bars = reinterpret_cast<Bars*>(base + kQBytes + kRingBytes);
   volatile int* abort_flag = &bars->abort;
+  // the leader CTA's copy of a barrier (cluster address)
+  auto lead = [&](uint64_t* bar) -> uint32_t { return mapa_shared(smem_u32(bar), 0); };
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->q_full[i]), 1);
+      mbar_init(smem_u32(&bars->q_empty[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_full[i]), 8);
+      mbar_init(smem_u32(&bars->o_full[i]), 1);
+      mbar_init(smem_u32(&bars->o_empty[i]), 8);
+    }
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->p_full[i]), kSubRows);
-      mbar_init(smem_u32(&bars->o_full[i]), 1);
     }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
   if (warp == 9) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint64_t tlim = p.timeout_ns;
+  const int causal = p.causal;
+  const int num_tiles = p.ws->num_tiles;
+  const int num_entries = p.ws->num_entries;
+  auto wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
+    return mbar_wait_cluster(bar, parity, abort_flag, err, tlim);
+  };
 
   if (warp == 8) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0 && nblk > 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
-      const uint32_t qbar = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qbar, kQBytes);
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int c = 0; c < kQkChunks; ++c)
-          tma_load_2d_hint(sQ + (i * kQkChunks + c) * kChunkBytes, &tm_q, h * kDqk + 64 * c,
-                           q_start + m0 + i * kSubRows, qbar, pol_q);
-      int issued = 0;
+      int item = 0;  // ring units issued so far
       bool ok = true;
-      for (int n = 0; n < nblk && ok; ++n) {
-        for (int it = 0; it < kItemsPerBlock; ++it) {
-          const int item = n * kItemsPerBlock + it;
-          const int slot = item % kRing;
-          const uint32_t round = static_cast<uint32_t>(item / kRing);
-          if (!mbar_wait(smem_u32(&bars->empty[slot]), (round & 1u) ^ 1u, abort_flag,
-                         MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim)) {
-            ok = false;
+      for (int k = 0; ok; ++k) {
+        const TileInfo ti = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
+        if (!ti.valid) break;
+        int nb[2];
+        tile_blocks(ti, causal, nb);
+        const int nblk = max(nb[0], nb[1]);
+        // Q rows of this CTA, once the previous tile's last S MMA has read them.
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (!(ok = wait(smem_u32(&bars->q_empty[i]), (static_cast<uint32_t>(k) & 1u) ^ 1u,
+                          MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
+          if (nb[i] > 0) {
+            if (leader) mbar_arrive_expect_tx(smem_u32(&bars->q_full[i]), 2 * kQSubBytes);
+            const uint32_t qbar = lead(&bars->q_full[i]);
+#pragma unroll
+            for (int c = 0; c < kQkChunks; ++c)
+              tma_load_2d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q,
+                               ti.h * kDqk + 64 * c,
+                               ti.q_start + ti.m0 + i * kSubRows + static_cast<int>(rank) * kCtaRows,
+                               qbar, pol_q);
+          } else if (leader) {
+            mbar_arrive(smem_u32(&bars->q_full[i]));
           }
-          const uint32_t fbar = smem_u32(&bars->full[slot]);
-          mbar_arrive_expect_tx(fbar, kChunkBytes);
-          if (it < kQkChunks)
-            tma_load_2d_hint(sRing + slot * kChunkBytes, &tm_k, h * kDqk + 64 * it,
-                             k_start + n * kBlockKeys, fbar, pol_kv);
-          else
-            tma_load_2d_hint(sRing + slot * kChunkBytes, &tm_v, h * kDv + 64 * (it - kQkChunks),
-                             k_start + n * kBlockKeys, fbar, pol_kv);
-          ++issued;
+        }
+        for (int n = 0; n < nblk && ok; ++n) {
+          for (int it = 0; it < kItemsPerBlock; ++it, ++item) {
+            const int rslot = item % kRing;
+            if (!(ok = wait(smem_u32(&bars->empty[rslot]),
+                            (static_cast<uint32_t>(item / kRing) & 1u) ^ 1u,
+                            MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
+              break;
+            if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[rslot]), 2 * kUnitBytes);
+            const uint32_t fbar = lead(&bars->full[rslot]);
+            const int key0 = ti.k_start + n * kBlockKeys;
+            if (it < kKUnits)  // K: this CTA's 64 keys, 64 of the 192 dims
+              tma_load_2d_pair(sRing + rslot * kUnitBytes, &tm_k, ti.h * kDqk + 64 * it,
+                               key0 + static_cast<int>(rank) * kHalfKeys, fbar, pol_kv);
+            else  // V: 64 keys, this CTA's 64 of the 128 value dims
+              tma_load_2d_pair(sRing + rslot * kUnitBytes, &tm_v,
+                               ti.h * kDv + static_cast<int>(rank) * kHalfDv,
+                               key0 + 64 * (it - kKUnits), fbar, pol_kv);
+          }
         }
       }
-      if (!ok) {
+      if (!ok && leader) {
         // Unwinding: let the copies already issued land before the CTA exits.
         volatile int no_abort = 0;
-        mbar_wait(qbar, 0, &no_abort, 0, tlim);
-        const int first = max(0, issued - kRing);
-        for (int item = first; item < issued; ++item) {
-          mbar_wait(smem_u32(&bars->full[item % kRing]),
-                    static_cast<uint32_t>(item / kRing) & 1u, &no_abort, 0, tlim);
-        }
+        const int first = max(0, item - kRing);
+        for (int it = first; it < item; ++it)
+          mbar_wait_cluster(smem_u32(&bars->full[it % kRing]),
+                            static_cast<uint32_t>(it / kRing) & 1u, &no_abort, 0, tlim);
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------- MMA issuer
-    if (nblk > 0) {
-      auto wait_item = [&](int item) -> bool {
-        return __all_sync(0xffffffffu,
-                          mbar_wait(smem_u32(&bars->full[item % kRing]),
-                                    static_cast<uint32_t>(item / kRing) & 1u, abort_flag,
-                                    MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim));
-      };
-      auto release_item = [&](int item) {
-        if (lane == 0) tc_commit(smem_u32(&bars->empty[item % kRing]));
-      };
-      auto issue_s = [&](int i, int n) {
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < kDqk / 16; ++kk) {
-            const int c = kk >> 2;
-            const uint32_t koff = (kk & 3) * 32;
-            const uint64_t a = sdesc_sw128(sQ + (i * kQkChunks + c) * kChunkBytes + koff, 16, 1024);
-            const int slot = (n * kItemsPerBlock + c) % kRing;
-            const uint64_t bd = sdesc_sw128(sRing + slot * kChunkBytes + koff, 16, 1024);
-            mma_ss(tmem + i * 128, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&bars->s_full[i]));
-        }
-        __syncwarp();
-      };
-      auto issue_pv = [&](int i, int n) {
-        if (lane == 0) {
-          const int slot0 = (n * kItemsPerBlock + kQkChunks) % kRing;
-          const int slot1 = (n * kItemsPerBlock + kQkChunks + 1) % kRing;
-          const uint32_t tO = tmem + 256 + i * 128;
-#pragma unroll
-          for (int kk = 0; kk < kBlockKeys / 16; ++kk) {
-            const uint32_t a_t = tmem + i * 128 + kk * 8;  // 16 bf16 of P = 8 columns
-            const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-            const uint32_t koff = kk * 16 * 128;           // 16 key rows of 128 bytes
-            if (slot1 == slot0 + 1) {
-              const uint64_t bd = sdesc_sw128(sRing + slot0 * kChunkBytes + koff, kChunkBytes, 1024);
-              mma_ts(tO, a_t, bd, kIdescPV128, acc);
-            } else {
-              const uint64_t b0 = sdesc_sw128(sRing + slot0 * kChunkBytes + koff, kChunkBytes, 1024);
-              const uint64_t b1 = sdesc_sw128(sRing + slot1 * kChunkBytes + koff, kChunkBytes, 1024);
-              mma_ts(tO, a_t, b0, kIdescPV64, acc);
-              mma_ts(tO + 64, a_t, b1, kIdescPV64, acc);
-            }
-          }
-        }
-        __syncwarp();
-      };
-      auto wait_p = [&](int i, int n) -> bool {
-        const bool ok = __all_sync(0xffffffffu,
-                                   mbar_wait(smem_u32(&bars->p_full[i]), static_cast<uint32_t>(n) & 1u,
-                                             abort_flag, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim));
+    // -------------------------------------------- MMA issuer (leader only)
+    if (leader) {
+      bool ok = true;
+      auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+        const bool r = __all_sync(0xffffffffu, wait(bar, parity, MLA_DEVSTAT_WAIT_TIMEOUT_MMA));
         tc_fence_after();
-        return ok;
+        return r;
+      };
+      auto wait_item = [&](int item) -> bool {
+        return wait_bar(smem_u32(&bars->full[item % kRing]),
+                        static_cast<uint32_t>(item / kRing) & 1u);
+      };
+      auto commit_both = [&](uint64_t* bar) { tc_commit_pair_elect(smem_u32(bar), 0x3); };
+      auto release_item = [&](int item) { commit_both(&bars->empty[item % kRing]); };
+      auto issue_s = [&](int i, int kitem) {
+#pragma unroll
+        for (int kk = 0; kk < kDqk / 16; ++kk) {
+          const int c = kk >> 2;
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t a =
+              sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes + koff, 16, 1024);
+          const uint64_t bd =
+              sdesc_sw128(sRing + ((kitem + c) % kRing) * kUnitBytes + koff, 16, 1024);
+          mma2_ss_elect(tmem + i * 128, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        commit_both(&bars->s_full[i]);
+      };
+      auto issue_pv = [&](int i, int vitem, bool first) {
+        const uint32_t tO = tmem + 256 + i * 128;
+#pragma unroll
+        for (int kk = 0; kk < kBlockKeys / 16; ++kk) {
+          const uint32_t a_t = tmem + i * 128 + kk * 8;  // 16 bf16 of P = 8 columns
+          const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+          const int unit = (vitem + (kk >> 2)) % kRing;  // 64 keys per unit
+          const uint64_t bd =
+              sdesc_sw128(sRing + unit * kUnitBytes + (kk & 3) * 16 * 128, kUnitBytes, 1024);
+          mma2_ts_elect(tO, a_t, bd, kIdescPV, acc);
+        }
       };
 
-      bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->q_full), 0, abort_flag,
-                                                  MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim));
-      for (int c = 0; c < kQkChunks && ok; ++c) ok = wait_item(c);
-      if (ok) {
-        tc_fence_after();
-        if (nb0 > 0) issue_s(0, 0);
-        if (nb1 > 0) issue_s(1, 0);
-        for (int c = 0; c < kQkChunks; ++c) release_item(c);
-      }
-      for (int n = 0; n < nblk && ok; ++n) {
-        const int vbase = n * kItemsPerBlock + kQkChunks;
-        ok = wait_item(vbase) && wait_item(vbase + 1);
+      int item = 0;           // first ring unit of the current tile
+      int p_cnt[2] = {0, 0};  // P blocks consumed per sub-tile (p_full parity)
+      int o_cnt[2] = {0, 0};  // O-using tiles per sub-tile (o_full / o_empty parity)
+      // First S MMAs of a tile when the previous tile did not issue them.
+      auto start_tile = [&](const int (&n)[2], int kitem, int k) -> bool {
+        for (int i = 0; i < 2; ++i)
+          if (!wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k) & 1u)) return false;
+        if (max(n[0], n[1]) > 0) {
+          for (int c = 0; c < kKUnits; ++c)
+            if (!wait_item(kitem + c)) return false;
+          for (int i = 0; i < 2; ++i) {
+            if (n[i] > 0) issue_s(i, kitem);
+            if (n[i] <= 1) commit_both(&bars->q_empty[i]);
+          }
+          for (int c = 0; c < kKUnits; ++c) release_item(kitem + c);
+        } else {
+          for (int i = 0; i < 2; ++i) commit_both(&bars->q_empty[i]);
+        }
+        return true;
+      };
+
+      int k = 0;
+      TileInfo cur = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
+      int nb[2];
+      tile_blocks(cur, causal, nb);
+      if (cur.valid) ok = start_tile(nb, item, k);
+      while (ok && cur.valid) {
+        const int nblk = max(nb[0], nb[1]);
+        const TileInfo nxt = tile_at(p, k + 1, cluster, nclusters, num_tiles, num_entries);
+        int nbn[2];
+        tile_blocks(nxt, causal, nbn);
+        for (int n = 0; n < nblk && ok; ++n) {
+          const int vitem = item + n * kItemsPerBlock + kKUnits;
+          const bool last = n + 1 == nblk;
+          if (!(ok = wait_item(vitem) && wait_item(vitem + 1))) break;
+          // The next KV block is (cur, n+1), or block 0 of the next tile.
+          const int kitem_next = item + (n + 1) * kItemsPerBlock;
+          bool next_s[2] = {n + 1 < nb[0], n + 1 < nb[1]};
+          if (last) {
+            next_s[0] = nbn[0] > 0;
+            next_s[1] = nbn[1] > 0;
+          }
+          const bool more = next_s[0] || next_s[1];
+          if (more && !(ok = wait_item(kitem_next) && wait_item(kitem_next + 1) &&
+                             wait_item(kitem_next + 2)))
+            break;
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (n < nb[i]) {
+              if (n == 0 && !(ok = wait_bar(smem_u32(&bars->o_empty[i]),
+                                            (static_cast<uint32_t>(o_cnt[i]) & 1u) ^ 1u)))
+                break;
+              if (!(ok = wait_bar(smem_u32(&bars->p_full[i]),
+                                  static_cast<uint32_t>(p_cnt[i]) & 1u)))
+                break;
+              ++p_cnt[i];
+              issue_pv(i, vitem, n == 0);
+              if (n == nb[i] - 1) {
+                commit_both(&bars->o_full[i]);
+                ++o_cnt[i];
+              }
+            }
+            if (i == 1) {  // both PVs of block n issued: V(n) can be refilled
+              release_item(vitem);
+              release_item(vitem + 1);
+            }
+            if (last && nxt.valid &&
+                !(ok = wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k + 1) & 1u)))
+              break;
+            if (next_s[i]) {
+              issue_s(i, kitem_next);
+              // Q_i is free after the last S MMA of its tile
+              const int nbi = last ? nbn[i] : nb[i];
+              const int nidx = last ? 0 : n + 1;
+              if (nidx == nbi - 1) commit_both(&bars->q_empty[i]);
+            } else if (last && nxt.valid) {
+              commit_both(&bars->q_empty[i]);  // no S for it in the next tile
+            }
+          }
+          if (ok && more)
+            for (int c = 0; c < kKUnits; ++c) release_item(kitem_next + c);
+        }
         if (!ok) break;
-        tc_fence_after();
-        if (n < nb0) {
-          if (!(ok = wait_p(0, n))) break;
-          issue_pv(0, n);
-          if (n == nb0 - 1 && lane == 0) tc_commit(smem_u32(&bars->o_full[0]));
-        }
-        const bool more = n + 1 < nblk;
-        if (more) {
-          const int kbase = (n + 1) * kItemsPerBlock;
-          ok = wait_item(kbase) && wait_item(kbase + 1) && wait_item(kbase + 2);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        if (n + 1 < nb0) issue_s(0, n + 1);
-        if (n < nb1) {
-          if (!(ok = wait_p(1, n))) break;
-          issue_pv(1, n);
-          if (n == nb1 - 1 && lane == 0) tc_commit(smem_u32(&bars->o_full[1]));
-        }
-        if (more) {
-          release_item(vbase);
-          release_item(vbase + 1);
-        }
-        if (n + 1 < nb1) issue_s(1, n + 1);
-        if (more) {
-          const int kbase = (n + 1) * kItemsPerBlock;
-          for (int c = 0; c < kQkChunks; ++c) release_item(kbase + c);
-        }
+        if (nblk == 0 && nxt.valid && !(ok = start_tile(nbn, item, k + 1))) break;
+        item += nblk * kItemsPerBlock;
+        ++k;
+        cur = nxt;
+        nb[0] = nbn[0];
+        nb[1] = nbn[1];
       }
-      // Wait until every MMA issued above has completed before the CTA ends.
-      if (lane == 0) tc_commit(smem_u32(&bars->drain));
+      // Wait until every MMA issued above has completed.
+      tc_commit_pair_elect(smem_u32(&bars->drain), 0x1);
       __syncwarp();
       volatile int no_abort = 0;
-      mbar_wait(smem_u32(&bars->drain), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
+      mbar_wait_cluster(smem_u32(&bars->drain), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
     }
   } else {
-    // ------------------------------------------------- softmax warpgroups
+    // ------------------------------------------------ softmax warpgroups
     const int sub = warp >> 2;
     const int wq = warp & 3;
-    const int r = m0 + sub * kSubRows + wq * 32 + lane;  // row within the sequence
-    const int row0 = m0 + sub * kSubRows;
-    const int nb = sub == 0 ? nb0 : nb1;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + sub * 128;
     const uint32_t tO = tmem + lane_off + 256 + sub * 128;
-    const int lim = p.causal ? min(Lk, r + off + 1) : Lk;  // keys [0, lim) visible
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
-    float l_run = 0.f;        // running sum of exp2(scaled s - m_run)
-    bool ok = true;
     const uint32_t sbar = smem_u32(&bars->s_full[sub]);
-    const uint32_t pbar = smem_u32(&bars->p_full[sub]);
+    const uint32_t pbar_lead = lead(&bars->p_full[sub]);
+    const uint32_t obar_lead = lead(&bars->o_empty[sub]);
+    int s_cnt = 0;  // S blocks consumed (s_full parity)
+    int o_cnt = 0;  // O-using tiles (o_full parity)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const TileInfo ti = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
+      if (!ti.valid) break;
+      const int row0 = ti.m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows;  // this CTA's rows
+      const int r = row0 + wq * 32 + lane;  // row within the sequence
+      const int off = ti.Lk - ti.Lq;
+      const int nb = blocks_for(sub_tile_keys(ti.m0 + sub * kSubRows, ti.Lq, ti.Lk, causal));
+      const int lim = causal ? min(ti.Lk, r + off + 1) : ti.Lk;  // keys [0, lim) visible
+      float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
+      float l_run = 0.f;        // running sum of exp2(scaled s - m_run)
 
-    for (int n = 0; n < nb; ++n) {
-      ok = __all_sync(0xffffffffu, mbar_wait(sbar, static_cast<uint32_t>(n) & 1u, abort_flag,
-                                             MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX, tlim));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sraw[128];
-      tmem_ld_x128_wait(tS, sraw);
-      float x[128];
+      for (int n = 0; n < nb; ++n) {
+        ok = __all_sync(0xffffffffu, wait(sbar, static_cast<uint32_t>(s_cnt) & 1u,
+                                          MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX));
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sraw[128];
+        tmem_ld_x128_wait(tS, sraw);
+        float x[128];
 #pragma unroll
-      for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(sraw[j]);
-      const int kbase = n * kBlockKeys;
-      const bool full_blk = (kbase + kBlockKeys <= Lk) &&
-                            (!p.causal || kbase + kBlockKeys - 1 <= row0 + off);
-      if (!full_blk) {
+        for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(sraw[j]);
+        const int kbase = n * kBlockKeys;
+        const bool full_blk = (kbase + kBlockKeys <= ti.Lk) &&
+                              (!causal || kbase + kBlockKeys - 1 <= row0 + off);
+        if (!full_blk) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (kbase + j >= lim) x[j] = -INFINITY;
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int j = 1; j < 128; ++j) mx = fmaxf(mx, x[j]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      // Lazy rescaling: keep the old maximum unless the new one is larger by
-      // more than 8 (a factor 256 in the exponentials, harmless in fp32/bf16).
-      const bool need = m_new > m_run + 8.0f;
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ex2_approx(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-      float sum = 0.0f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {  // 32 scores -> 16 packed bf16 pairs per store
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = ex2_approx(fmaf(x[32 * c + 2 * j], sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(x[32 * c + 2 * j + 1], sl2, -m_use));
-          sum += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
+          for (int j = 0; j < 128; ++j)
+            if (kbase + j >= lim) x[j] = -INFINITY;
         }
-        tmem_st_x16(tS + 16u * c, pk);
+        float m8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+        for (int j = 8; j < 128; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        // Lazy rescaling: keep the old maximum unless the new one is larger by
+        // more than 8 (a factor 256 in the exponentials, harmless in fp32/bf16).
+        const bool need = m_new > m_run + 8.0f;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 32 scores -> 16 packed bf16 pairs per store
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p0 = ex2_approx(fmaf(x[32 * c + 2 * j], sl2, -m_use));
+            const float p1 = ex2_approx(fmaf(x[32 * c + 2 * j + 1], sl2, -m_use));
+            sum4[j & 3] += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x16(tS + 16u * c, pk);
+        }
+        l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        // O(n-1) is complete (its MMAs precede S(n) in issue order) and PV(n)
+        // waits for p_full, so O can be rescaled here, after the scores died.
+        if (n > 0 && __any_sync(0xffffffffu, need)) rescale_o_row(tO, alpha);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(pbar_lead);
       }
-      l_run += sum;
-      // O(n-1) is complete (its MMAs precede S(n) in issue order) and PV(n)
-      // waits for p_full, so O can be rescaled here, after the scores died.
-      if (n > 0 && __any_sync(0xffffffffu, need)) rescale_o_row(tO, alpha);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(pbar);
-    }
+      if (!ok) break;
 
-    // --------------------------------------------------------- epilogue
-    const bool row_ok = r < Lq;
-    const size_t row_index = static_cast<size_t>(q_start + r) * p.num_heads + h;
-    uint4* orow = reinterpret_cast<uint4*>(p.out + row_index * kDv);
-    float lse_val = -INFINITY;
-    if (nb > 0 && ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full[sub]), 0, abort_flag,
-                                             MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX, tlim));
-    }
-    if (nb > 0 && ok) {
-      tc_fence_after();
-      const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld_x32_wait(tO + 32u * c, o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
+      // ------------------------------------------------------- epilogue
+      const bool row_ok = r < ti.Lq;
+      const size_t row_index = static_cast<size_t>(ti.q_start + r) * p.num_heads + ti.h;
+      uint4* orow = reinterpret_cast<uint4*>(p.out + row_index * kDv);
+      float lse_val = -INFINITY;
+      if (nb > 0) {
+        ok = __all_sync(0xffffffffu, wait(smem_u32(&bars->o_full[sub]),
+                                          static_cast<uint32_t>(o_cnt) & 1u,
+                                          MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t o[128];
+        tmem_ld_x128_wait(tO, o);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(obar_lead);  // O may be overwritten now
+        ++o_cnt;
+        const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
         if (row_ok) {
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-      if (l_run > 0.0f) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
-    } else if (row_ok) {
+          for (int v4 = 0; v4 < 16; ++v4) {
+            uint32_t pk[4];
 #pragma unroll
-      for (int v4 = 0; v4 < 16; ++v4) orow[v4] = make_uint4(0u, 0u, 0u, 0u);
+            for (int j = 0; j < 4; ++j)
+              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
+                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv);
+            orow[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        if (l_run > 0.0f) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
+      } else if (row_ok) {
+#pragma unroll
+        for (int v4 = 0; v4 < 16; ++v4) orow[v4] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (row_ok && p.lse != nullptr)
+        p.lse[static_cast<size_t>(ti.h) * p.total_q + ti.q_start + r] = lse_val;
     }
-    if (row_ok && p.lse != nullptr) p.lse[static_cast<size_t>(h) * p.total_q + q_start + r] = lse_val;
   }
 
+  // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still
+  // read its shared memory or write its TMEM.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 

@@ -12,7 +12,7 @@
 #include <cstdlib>
 #include <mutex>
 
-#include "../../include/mla.h"
+#include "mla.h"
 #include "dense_fwd.cuh"
 #include "merge.cuh"
 
@@ -57,6 +57,8 @@ struct DeviceState {
   int checked = 0;  // 0 unknown, 1 ok, -1 unsupported
 };
 DeviceState g_dev[kMaxDevices];
+int g_dev_sms[kMaxDevices];
+int g_dev_dense_clusters[kMaxDevices];  // co-resident 2-CTA clusters of the dense kernel
 std::mutex g_dev_mu;
 
 int prepare_device(int* dev_out) {
@@ -81,6 +83,26 @@ int prepare_device(int* dev_out) {
                            mla::dense::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (encode_fn() == nullptr) return MLA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2), 1, 1);
+    cfg.blockDim = dim3(mla::dense::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = mla::dense::kSmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mla::dense::dense_fwd_kernel, &cfg) != cudaSuccess ||
+        n < 1)
+      return MLA_ERR_CUDA;
+    g_dev_dense_clusters[dev] = n;
+  }
   g_dev[dev].checked = 1;
   return MLA_OK;
 }
@@ -88,12 +110,13 @@ int prepare_device(int* dev_out) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix with a
-// 64-column x 128-row box and the 128-byte swizzle.  Rows past `rows` read
+// 64-column x box_rows box and the 128-byte swizzle.  Rows past `rows` read
 // as zero.
-int encode_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+int encode_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                uint32_t box_rows) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
                                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -139,46 +162,87 @@ const char* mla_status_string(int status) {
 
 int mla_version(void) { return 100; }
 
+size_t mla_prefill_workspace_size(int batch, int total_q) {
+  if (batch < 1 || total_q < 0) return 0;
+  const size_t entries = static_cast<size_t>((total_q + mla::dense::kTileRows - 1) /
+                                             mla::dense::kTileRows) + static_cast<size_t>(batch);
+  return mla::dense::kWsHeaderBytes + entries * sizeof(int2);
+}
+
 int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
                     const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
                     float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
-                    int batch, int num_heads, int total_q, int total_k) {
+                    int batch, int num_heads, int total_q, int total_k, void* workspace,
+                    size_t workspace_bytes) {
   using namespace mla::dense;
   if (q == nullptr || k == nullptr || v == nullptr || cu_seqlens_q == nullptr ||
-      cu_seqlens_k == nullptr || out == nullptr)
+      cu_seqlens_k == nullptr || out == nullptr || workspace == nullptr)
     return MLA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || (lse && !aligned(lse, 4)))
+      !aligned(workspace, 16) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      (lse && !aligned(lse, 4)))
     return MLA_ERR_INVALID_ARG;
-  if (batch < 1 || batch > 65535 || num_heads < 1 || num_heads > 65535 || total_q < 0 ||
-      total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || (causal != 0 && causal != 1))
+  if (batch < 1 || num_heads < 1 || num_heads > 65535 || total_q < 0 || total_k < 0 ||
+      max_seqlen_q < 0 || max_seqlen_k < 0 || (causal != 0 && causal != 1))
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_prefill_workspace_size(batch, total_q);
+  if (workspace_bytes < need) return MLA_ERR_INVALID_ARG;
   int dev = 0;
   int st = prepare_device(&dev);
   if (st != MLA_OK) return st;
-  if (total_q == 0 || max_seqlen_q == 0) return MLA_OK;  // nothing to compute
+  if (total_q == 0) return MLA_OK;  // nothing to compute
 
   CUtensorMap tq, tk, tv;
   const uint64_t kv_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
-  if ((st = encode_rows(&tq, q, static_cast<uint64_t>(num_heads) * kDqk, total_q)) != MLA_OK ||
-      (st = encode_rows(&tk, k, static_cast<uint64_t>(num_heads) * kDqk, kv_rows)) != MLA_OK ||
-      (st = encode_rows(&tv, v, static_cast<uint64_t>(num_heads) * kDv, kv_rows)) != MLA_OK)
+  if ((st = encode_rows(&tq, q, static_cast<uint64_t>(num_heads) * kDqk, total_q, kCtaRows)) !=
+          MLA_OK ||
+      (st = encode_rows(&tk, k, static_cast<uint64_t>(num_heads) * kDqk, kv_rows, kHalfKeys)) !=
+          MLA_OK ||
+      (st = encode_rows(&tv, v, static_cast<uint64_t>(num_heads) * kDv, kv_rows, 64)) != MLA_OK)
     return st;
+
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* ws = static_cast<WsHeader*>(workspace);
+  int2* entries = reinterpret_cast<int2*>(static_cast<char*>(workspace) + kWsHeaderBytes);
+  const int capacity = static_cast<int>((need - kWsHeaderBytes) / sizeof(int2));
+  dense_plan_kernel<<<1, kPlanThreads, 0, s>>>(cu_seqlens_q, cu_seqlens_k, batch, causal, ws,
+                                               entries, capacity, num_heads);
+  if ((st = launch_status()) != MLA_OK) return st;
 
   Params p;
   p.cu_q = cu_seqlens_q;
   p.cu_k = cu_seqlens_k;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.ws = ws;
+  p.entries = entries;
   p.num_heads = num_heads;
   p.total_q = total_q;
   p.causal = causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
   p.timeout_ns = wait_timeout_ns();
-  const dim3 grid((max_seqlen_q + kCtaRows - 1) / kCtaRows, num_heads, batch);
-  dense_fwd_kernel<<<grid, kThreads, kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk,
-                                                                                       tv, p);
+  // Persistent: as many 2-CTA clusters as can be resident at once, but never
+  // more than tiles could exist.
+  const long long max_tiles = static_cast<long long>(capacity) * num_heads;
+  const long long clusters =
+      max_tiles < g_dev_dense_clusters[dev] ? max_tiles : g_dev_dense_clusters[dev];
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dense_fwd_kernel, tq, tk, tv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
   return launch_status();
 }
 

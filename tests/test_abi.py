@@ -42,18 +42,27 @@ def test_status_strings_and_version():
 
 def _call_dense(**over):
     a = dict(q=16, k=16, v=16, cq=16, ck=16, mq=4, mk=4, scale=0.1, causal=1, out=16, lse=None,
-             stream=None, batch=1, H=1, tq=4, tk=4)
+             stream=None, batch=1, H=1, tq=4, tk=4, ws=64, wsb=4096)
     a.update(over)
     P = lambda x: None if x is None else ctypes.c_void_p(x)
     return mla.load().mla_prefill_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["cq"]), P(a["ck"]),
                                       a["mq"], a["mk"], a["scale"], a["causal"], P(a["out"]),
-                                      P(a["lse"]), None, a["batch"], a["H"], a["tq"], a["tk"])
+                                      P(a["lse"]), None, a["batch"], a["H"], a["tq"], a["tk"],
+                                      P(a["ws"]), a["wsb"])
+
+
+def test_workspace_size():
+    f = mla.prefill_workspace_size
+    assert f(1, 0) == 256 + 8 * 1  # header + one entry per (sequence, 512-row block)
+    assert f(8, 15843) == 256 + 8 * (31 + 8)
+    assert mla.load().mla_prefill_workspace_size(0, 10) == 0
 
 
 @pytest.mark.parametrize("over", [dict(q=None), dict(out=None), dict(cq=None), dict(q=24),
                                   dict(out=8), dict(cq=2), dict(batch=0), dict(H=0),
                                   dict(tq=-1), dict(causal=2), dict(scale=0.0),
-                                  dict(scale=float("nan")), dict(scale=-1.0), dict(lse=2)])
+                                  dict(scale=float("nan")), dict(scale=-1.0), dict(lse=2),
+                                  dict(ws=None), dict(ws=8), dict(wsb=100)])
 def test_dense_rejects_bad_arguments(over):
     assert _call_dense(**over) == _lib.MLA_ERR_INVALID_ARG
 

@@ -23,7 +23,7 @@
 // pair derive the same tile sequence without talking, clusters running at
 // the same time share K/V in L2, and the short tiles come last.
 //
-// Roles inside each CTA (320 threads):
+// Roles inside each CTA (384 threads):
 //   warps 0-3  softmax + epilogue, sub-tile 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax + epilogue, sub-tile 1
 //   warp  8    producer: TMA loads of this CTA's Q rows and K/V halves, whose
@@ -66,7 +66,15 @@ constexpr int kRing = 16;
 constexpr int kQSubBytes = kQkChunks * kQChunkBytes; // 48 KB
 constexpr int kQBytes = 2 * kQSubBytes;              // 96 KB
 constexpr int kRingBytes = kRing * kUnitBytes;       // 128 KB
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;          // 3 warpgroups; warps 10-11 only hold registers
+// Register split (setmaxnreg): launched at kLaunchRegs per thread, the two
+// softmax warpgroups grow to kSoftmaxRegs and the producer/MMA warpgroup
+// shrinks to kOtherRegs; 8*32*224 + 4*32*56 = 384*168, the launch's total.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kTmemCols = 512;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBins = 4096;                      // work histogram bins (clamped)
@@ -273,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     return mbar_wait_cluster(bar, parity, abort_flag, err, tlim);
   };
 
+  if (warp >= 8) {
+    setmaxnreg_dec<kOtherRegs>();
   if (warp == 8) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
@@ -351,29 +361,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto commit_both = [&](uint64_t* bar) { tc_commit_pair_elect(smem_u32(bar), 0x3); };
       auto release_item = [&](int item) { commit_both(&bars->empty[item % kRing]); };
+      // Descriptors: built once per burst, then advanced by adding to the
+      // start-address field (bits 0..13, in 16-byte units); no field carries
+      // since every operand lies below 256 KB of shared memory.
       auto issue_s = [&](int i, int kitem) {
+#pragma unroll 1
+        for (int c = 0; c < kQkChunks; ++c) {
+          uint64_t a = sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes, 16, 1024);
+          uint64_t bd = sdesc_sw128(sRing + ((kitem + c) % kRing) * kUnitBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kDqk / 16; ++kk) {
-          const int c = kk >> 2;
-          const uint32_t koff = (kk & 3) * 32;
-          const uint64_t a =
-              sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes + koff, 16, 1024);
-          const uint64_t bd =
-              sdesc_sw128(sRing + ((kitem + c) % kRing) * kUnitBytes + koff, 16, 1024);
-          mma2_ss_elect(tmem + i * 128, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {  // 16 dims (32 bytes) per MMA
+            mma2_ss_elect(tmem + i * 128, a, bd, kIdescQK, (c > 0 || kk > 0) ? 1u : 0u);
+            a += 2;
+            bd += 2;
+          }
         }
         commit_both(&bars->s_full[i]);
       };
       auto issue_pv = [&](int i, int vitem, bool first) {
         const uint32_t tO = tmem + 256 + i * 128;
+#pragma unroll 1
+        for (int u = 0; u < kVUnits; ++u) {  // 64 keys per unit
+          uint64_t bd = sdesc_sw128(sRing + ((vitem + u) % kRing) * kUnitBytes, kUnitBytes, 1024);
+          uint32_t a_t = tmem + i * 128 + u * 32;  // 16 bf16 of P = 8 columns per MMA
 #pragma unroll
-        for (int kk = 0; kk < kBlockKeys / 16; ++kk) {
-          const uint32_t a_t = tmem + i * 128 + kk * 8;  // 16 bf16 of P = 8 columns
-          const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-          const int unit = (vitem + (kk >> 2)) % kRing;  // 64 keys per unit
-          const uint64_t bd =
-              sdesc_sw128(sRing + unit * kUnitBytes + (kk & 3) * 16 * 128, kUnitBytes, 1024);
-          mma2_ts_elect(tO, a_t, bd, kIdescPV, acc);
+          for (int kk = 0; kk < 4; ++kk) {  // 16 keys (16 rows of 128 bytes) per MMA
+            mma2_ts_elect(tO, a_t, bd, kIdescPV, (!first || u > 0 || kk > 0) ? 1u : 0u);
+            a_t += 8;
+            bd += 128;
+          }
         }
       };
 
@@ -472,7 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait_cluster(smem_u32(&bars->drain), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
     }
+  }
   } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------ softmax warpgroups
     const int sub = warp >> 2;
     const int wq = warp & 3;
@@ -480,6 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + sub * 128;
     const uint32_t tO = tmem + lane_off + 256 + sub * 128;
     const float sl2 = p.scale_log2;
+    const uint64_t c2 = pack_f32x2(sl2, sl2);
+    const Exp2PolyConsts pk2 = exp2_poly_consts();
     const uint32_t sbar = smem_u32(&bars->s_full[sub]);
     const uint32_t pbar_lead = lead(&bars->p_full[sub]);
     const uint32_t obar_lead = lead(&bars->o_empty[sub]);
@@ -495,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nb = blocks_for(sub_tile_keys(ti.m0 + sub * kSubRows, ti.Lq, ti.Lk, causal));
       const int lim = causal ? min(ti.Lk, r + off + 1) : ti.Lk;  // keys [0, lim) visible
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
-      float l_run = 0.f;        // running sum of exp2(scaled s - m_run)
+      float l_run = 0.f;        // running sum of the fp32 weights exp2(scaled s - m_run)
 
       for (int n = 0; n < nb; ++n) {
         ok = __all_sync(0xffffffffu, wait(sbar, static_cast<uint32_t>(s_cnt) & 1u,
@@ -518,11 +538,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float m8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m8[j] = x[j];
+        for (int t = 0; t < 8; ++t) m8[t] = x[t];
 #pragma unroll
-        for (int j = 8; j < 128; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int j = 8; j < 120; j += 16)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) m8[t] = fmax3(m8[t], x[j + t], x[j + 8 + t]);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) m8[t] = fmaxf(m8[t], x[120 + t]);
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
         const float m_new = fmaxf(m_run, mx * sl2);
         // Lazy rescaling: keep the old maximum unless the new one is larger by
         // more than 8 (a factor 256 in the exponentials, harmless in fp32/bf16).
@@ -534,20 +558,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = m_new;
         }
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 32 scores -> 16 packed bf16 pairs per store
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float p0 = ex2_approx(fmaf(x[32 * c + 2 * j], sl2, -m_use));
-            const float p1 = ex2_approx(fmaf(x[32 * c + 2 * j + 1], sl2, -m_use));
-            sum4[j & 3] += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
+            // 10 of every 16 pairs on the MUFU unit, 6 on the FMA pipe
+            if ((j & 7) < 5)
+              pk[j] = softmax_pair_mufu(x[32 * c + 2 * j], x[32 * c + 2 * j + 1], c2, negm2,
+                                        acc[j & 3]);
+            else
+              pk[j] = softmax_pair_poly(x[32 * c + 2 * j], x[32 * c + 2 * j + 1], c2, negm2, pk2,
+                                        acc[j & 3]);
           }
           tmem_st_x16(tS + 16u * c, pk);
         }
-        l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        l_run += (sum_f32x2(acc[0]) + sum_f32x2(acc[1])) + (sum_f32x2(acc[2]) + sum_f32x2(acc[3]));
         // O(n-1) is complete (its MMAs precede S(n) in issue order) and PV(n)
         // waits for p_full, so O can be rescaled here, after the scores died.
         if (n > 0 && __any_sync(0xffffffffu, need)) rescale_o_row(tO, alpha);
@@ -575,7 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(obar_lead);  // O may be overwritten now
         ++o_cnt;
-        const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        // A row that saw no key keeps m_run = -inf (its weights are only the
+        // tiny clamped values of the polynomial path): output 0, LSE -inf.
+        const bool seen = m_run != -INFINITY;
+        const float inv = seen ? 1.0f / l_run : 0.0f;
         if (row_ok) {
 #pragma unroll
           for (int v4 = 0; v4 < 16; ++v4) {
@@ -587,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             orow[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
-        if (l_run > 0.0f) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
+        if (seen) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
       } else if (row_ok) {
 #pragma unroll
         for (int v4 = 0; v4 < 16; ++v4) orow[v4] = make_uint4(0u, 0u, 0u, 0u);

@@ -82,6 +82,17 @@ int prepare_device(int* dev_out) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            mla::dense::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
+  {
+    // The kernel's setmaxnreg split assumes this launch register count; a
+    // different count could make the warps that grow wait for ever.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, mla::dense::dense_fwd_kernel) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (fa.numRegs != mla::dense::kLaunchRegs) {
+      g_dev[dev].checked = -1;
+      return MLA_ERR_UNSUPPORTED;
+    }
+  }
   if (encode_fn() == nullptr) return MLA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MLA_ERR_CUDA;

@@ -49,6 +49,23 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity)
       : "memory");
   return ok;
 }
+// try_wait that may suspend the thread (without using issue slots) for up to
+// kSuspendHintNs while the phase is incomplete; the hardware resumes it as
+// soon as the phase completes.
+constexpr uint32_t kSuspendHintNs = 200000;
+__device__ __forceinline__ uint32_t mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kSuspendHintNs)
+      : "memory");
+  return ok;
+}
 
 // Wait for the phase with the given parity to complete.  Returns false when
 // the wait gave up: either the time limit passed (the status word gets
@@ -57,15 +74,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           unsigned int err_bit, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        atomicOr(&g_mla_status, err_bit);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      atomicOr(&g_mla_status, err_bit);
+      return false;
     }
   }
 }
@@ -190,6 +205,17 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 
+// Per-warpgroup register reallocation (all four warps of the warpgroup
+// execute the same instruction).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -206,22 +232,38 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on an mbarrier that may live in another CTA of the cluster.
+// Arrive on an mbarrier that may live in another CTA of the cluster.  The
+// default (CTA-scope release) semantics suffice here: what the arrival
+// publishes is tcgen05 state (TMEM), which the arriving thread has ordered
+// with tcgen05.wait + tcgen05.fence::before_thread_sync and the waiting
+// thread orders with tcgen05.fence::after_thread_sync.  A cluster-scope
+// release would also wait for every earlier global store of the thread.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-__device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity,
+                                                       bool suspend) {
   uint32_t ok;
-  asm volatile(
-      "{\n"
-      ".reg .pred p;\n"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-      "selp.u32 %0, 1, 0, p;\n"
-      "}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if (suspend)
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(kSuspendHintNs)
+        : "memory");
+  else
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
   return ok;
 }
 // Bounded wait with cluster-scope acquire (for barriers that receive
@@ -229,17 +271,15 @@ __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
                                                   volatile int* abort, unsigned int err_bit,
                                                   uint64_t limit_ns) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  if (mbar_try_wait_cluster(bar, parity, false)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        atomicOr(&g_mla_status, err_bit);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_cluster(bar, parity, true)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      atomicOr(&g_mla_status, err_bit);
+      return false;
     }
   }
 }
@@ -373,6 +413,101 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)            // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N >> 3
          | (static_cast<uint32_t>(M >> 4) << 24);    // M >> 4
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Softmax weights for a pair of scores x0, x1 (scaled by log2(e) * scale):
+// t = x * c - m for both (packed fp32 FMA), p = 2^t in fp32; returns the
+// pair rounded to bf16 (element 0 in the low half) and adds the fp32 p
+// values to the packed accumulator `acc`.
+//
+// Two ways to get 2^t, so that the MUFU unit and the FMA pipe share the
+// work:
+//  * softmax_pair_mufu: the ex2.approx.ftz.f32 instruction;
+//  * softmax_pair_poly: Cody-Waite range reduction t = j + f, j = rint(t),
+//    f in [-1/2, 1/2] (the rounding is the add/subtract of 1.5 * 2^23),
+//    2^f from a cubic polynomial, and 2^j folded into the exponent field
+//    with an integer multiply-add.  The cubic minimises the maximum
+//    relative error on [-1/2, 1/2] (weighted least squares iterated to
+//    equal ripple, fitted offline in double precision): max relative error
+//    7.5e-5 over t in [-125, 8].  t is clamped at -125 first, so masked
+//    scores (-inf) give 2^-125 rather than 0; callers treat rows whose
+//    running maximum is still -inf as empty.
+__device__ __forceinline__ uint32_t softmax_pair_mufu(float x0, float x1, uint64_t c2, uint64_t negm2,
+                                                      uint64_t& acc) {
+  uint32_t pk;
+  asm("{\n"
+      ".reg .b64 xx, tt;\n"
+      ".reg .b32 a, b;\n"
+      "mov.b64 xx, {%2, %3};\n"
+      "fma.rn.f32x2 tt, xx, %4, %5;\n"
+      "mov.b64 {a, b}, tt;\n"
+      "ex2.approx.ftz.f32 a, a;\n"
+      "ex2.approx.ftz.f32 b, b;\n"
+      "cvt.rn.bf16x2.f32 %0, b, a;\n"
+      "mov.b64 tt, {a, b};\n"
+      "add.f32x2 %1, %1, tt;\n"
+      "}\n"
+      : "=r"(pk), "+l"(acc)
+      : "f"(x0), "f"(x1), "l"(c2), "l"(negm2));
+  return pk;
+}
+struct Exp2PolyConsts {
+  uint64_t magic2, c0, c1, c2, c3;  // each a packed pair of equal fp32 values
+};
+__device__ __forceinline__ uint64_t splat_f32x2(float v) {
+  return (static_cast<uint64_t>(__float_as_uint(v)) << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ Exp2PolyConsts exp2_poly_consts() {
+  Exp2PolyConsts k;
+  k.magic2 = splat_f32x2(12582912.0f);  // 1.5 * 2^23
+  k.c0 = splat_f32x2(0.9999280571937561f);
+  k.c1 = splat_f32x2(0.6932609677314758f);
+  k.c2 = splat_f32x2(0.24261115491390228f);
+  k.c3 = splat_f32x2(0.055171772837638855f);
+  return k;
+}
+__device__ __forceinline__ uint32_t softmax_pair_poly(float x0, float x1, uint64_t c2, uint64_t negm2,
+                                                      const Exp2PolyConsts& k, uint64_t& acc) {
+  uint32_t pk;
+  asm("{\n"
+      ".reg .b64 xx, tt, mg, jj, ff, pp;\n"
+      ".reg .b32 a, b, ta, tb, pa, pb;\n"
+      "mov.b64 xx, {%2, %3};\n"
+      "fma.rn.f32x2 tt, xx, %4, %5;\n"
+      "mov.b64 {a, b}, tt;\n"
+      "max.f32 a, a, 0fC2FA0000;\n"  // clamp at -125
+      "max.f32 b, b, 0fC2FA0000;\n"
+      "mov.b64 tt, {a, b};\n"
+      "add.rn.f32x2 mg, tt, %6;\n"   // t + 1.5*2^23: rint(t) in the low mantissa bits
+      "sub.rn.f32x2 jj, mg, %6;\n"   // rint(t)
+      "sub.rn.f32x2 ff, tt, jj;\n"   // f in [-1/2, 1/2]
+      "fma.rn.f32x2 pp, ff, %10, %9;\n"
+      "fma.rn.f32x2 pp, pp, ff, %8;\n"
+      "fma.rn.f32x2 pp, pp, ff, %7;\n"
+      "mov.b64 {pa, pb}, pp;\n"
+      "mov.b64 {ta, tb}, mg;\n"
+      "mad.lo.u32 pa, ta, 8388608, pa;\n"  // add rint(t) to the exponent field
+      "mad.lo.u32 pb, tb, 8388608, pb;\n"
+      "cvt.rn.bf16x2.f32 %0, pb, pa;\n"
+      "mov.b64 pp, {pa, pb};\n"
+      "add.f32x2 %1, %1, pp;\n"
+      "}\n"
+      : "=r"(pk), "+l"(acc)
+      : "f"(x0), "f"(x1), "l"(c2), "l"(negm2), "l"(k.magic2), "l"(k.c0), "l"(k.c1), "l"(k.c2),
+        "l"(k.c3));
+  return pk;
+}
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float sum_f32x2(uint64_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v)) + __uint_as_float(static_cast<uint32_t>(v >> 32));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -450,3 +450,28 @@ def test_row_subsets_match_full_evaluation():
     to, tl = oracle.sparse_prefill(s["q"], s["kv"], s["indices"], s["scale"], tokens=[5, 2])
     np.testing.assert_allclose(to, so[[5, 2]], rtol=0, atol=1e-13)
     np.testing.assert_allclose(tl, sl[:, [5, 2]], rtol=0, atol=1e-13)
+
+
+def test_exp2_polynomial_constants_error_bound():
+    """The cubic used by the kernel's FMA-pipe exp2 (Cody-Waite reduction to
+    f in [-1/2, 1/2], 2^rint(t) folded into the exponent) stays within 1e-4
+    relative error over t in [-125, 8], emulated step by step in float32."""
+    import re
+    src = open(ROOT_PTX).read()
+    block = src[src.index("Exp2PolyConsts exp2_poly_consts()"):]
+    c = [np.float32(float(v)) for v in re.findall(r"splat_f32x2\(([0-9.e+-]+)f\)", block)[1:5]]
+    x = np.linspace(-125, 8, 400001).astype(np.float32)
+    magic = np.float32(12582912.0)
+    t = (x + magic).astype(np.float32)
+    f = (x - (t - magic).astype(np.float32)).astype(np.float32)
+    p = c[3]
+    for k in (2, 1, 0):
+        p = (p * f + c[k]).astype(np.float32)
+    bits = (p.view(np.uint32).astype(np.uint64) + (t.view(np.uint32).astype(np.uint64) << 23))
+    res = (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32).astype(np.float64)
+    rel = np.abs(res / np.exp2(x.astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4
+
+
+ROOT_PTX = __import__("os").path.join(__import__("os").path.dirname(__import__("os").path.dirname(
+    __import__("os").path.abspath(__file__))), "mla_prefill_attention_causal_b200", "csrc", "ptx.cuh")

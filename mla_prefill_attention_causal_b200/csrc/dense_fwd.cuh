@@ -30,9 +30,11 @@
 //              completion is counted on the leader CTA's barriers
 //   warp  9    (leader CTA only) MMA issuer: S = Q K^T, O += P V
 // Shared memory per CTA: Q 96 KB (2 sub-tiles x 3 chunks of 128 rows x 64
-// dims) and a ring of 16 units of 8 KB (64 rows x 64 dims), all with the
-// 128-byte swizzle used by TMA and the MMA descriptors; one KV block takes
-// 5 units per CTA (3 for its K half, 2 for its V half).
+// dims), a K ring of 3 slots (this CTA's 64 keys x 192 dims = 3 units of
+// 64 rows x 64 dims, 24 KB) and a V ring of 3 slots (128 keys x this CTA's
+// 64 dims = 2 units, 16 KB), all with the 128-byte swizzle used by TMA and
+// the MMA descriptors.  One barrier per slot and direction: K(b) is freed
+// after both S MMAs of block b, V(b) after both PV MMAs.
 // TMEM per CTA (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1
 // [384,512); P_i (bf16, 64 columns) overwrites the first half of S_i.
 //
@@ -61,11 +63,12 @@ constexpr int kUnitBytes = 64 * 128;                 // 64 rows x 64 bf16
 constexpr int kQkChunks = kDqk / 64;                 // 3
 constexpr int kKUnits = kQkChunks;                   // K half: 64 keys x 192 dims
 constexpr int kVUnits = kBlockKeys / 64;             // V half: 128 keys x 64 dims
-constexpr int kItemsPerBlock = kKUnits + kVUnits;    // 5 ring units per KV block
-constexpr int kRing = 16;
+constexpr int kSlots = 3;                            // K and V blocks in flight per CTA
+constexpr int kKSlotBytes = kKUnits * kUnitBytes;    // 24 KB: this CTA's half of a K block
+constexpr int kVSlotBytes = kVUnits * kUnitBytes;    // 16 KB: this CTA's half of a V block
 constexpr int kQSubBytes = kQkChunks * kQChunkBytes; // 48 KB
 constexpr int kQBytes = 2 * kQSubBytes;              // 96 KB
-constexpr int kRingBytes = kRing * kUnitBytes;       // 128 KB
+constexpr int kRingBytes = kSlots * (kKSlotBytes + kVSlotBytes);  // 120 KB
 constexpr int kThreads = 384;          // 3 warpgroups; warps 10-11 only hold registers
 // Register split (setmaxnreg): launched at kLaunchRegs per thread, the two
 // softmax warpgroups grow to kSoftmaxRegs and the producer/MMA warpgroup
@@ -95,8 +98,10 @@ struct TileInfo {
 struct alignas(8) Bars {
   uint64_t q_full[2];    // leader: Q bytes of both CTAs
   uint64_t q_empty[2];   // both: last S MMA of the tile done
-  uint64_t full[kRing];  // leader: unit bytes of both CTAs
-  uint64_t empty[kRing]; // both: MMAs reading the unit done
+  uint64_t full_k[kSlots];   // leader: K-half bytes of both CTAs
+  uint64_t full_v[kSlots];   // leader: V-half bytes of both CTAs
+  uint64_t empty_k[kSlots];  // both: the S MMAs reading the K slot done
+  uint64_t empty_v[kSlots];  // both: the PV MMAs reading the V slot done
   uint64_t s_full[2];    // both
   uint64_t p_full[2];    // leader: 8 softmax warps (both CTAs)
   uint64_t o_full[2];    // both
@@ -242,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sQ = smem_u32(base);
-  const uint32_t sRing = sQ + kQBytes;
+  const uint32_t sRingK = sQ + kQBytes;                  // kSlots x 24 KB
+  const uint32_t sRingV = sRingK + kSlots * kKSlotBytes;  // kSlots x 16 KB
   Bars* bars = reinterpret_cast<Bars*>(base + kQBytes + kRingBytes);
   volatile int* abort_flag = &bars->abort;
   // the leader CTA's copy of a barrier (cluster address)
@@ -257,9 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->o_full[i]), 1);
       mbar_init(smem_u32(&bars->o_empty[i]), 8);
     }
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(smem_u32(&bars->full[i]), 1);
-      mbar_init(smem_u32(&bars->empty[i]), 1);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(smem_u32(&bars->full_k[i]), 1);
+      mbar_init(smem_u32(&bars->full_v[i]), 1);
+      mbar_init(smem_u32(&bars->empty_k[i]), 1);
+      mbar_init(smem_u32(&bars->empty_v[i]), 1);
     }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -291,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tm_v);
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
-      int item = 0;  // ring units issued so far
+      int blk = 0;  // KV blocks issued so far (slot = blk % kSlots)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const TileInfo ti = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
@@ -317,33 +325,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(smem_u32(&bars->q_full[i]));
           }
         }
-        for (int n = 0; n < nblk && ok; ++n) {
-          for (int it = 0; it < kItemsPerBlock; ++it, ++item) {
-            const int rslot = item % kRing;
-            if (!(ok = wait(smem_u32(&bars->empty[rslot]),
-                            (static_cast<uint32_t>(item / kRing) & 1u) ^ 1u,
-                            MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
-              break;
-            if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[rslot]), 2 * kUnitBytes);
-            const uint32_t fbar = lead(&bars->full[rslot]);
-            const int key0 = ti.k_start + n * kBlockKeys;
-            if (it < kKUnits)  // K: this CTA's 64 keys, 64 of the 192 dims
-              tma_load_2d_pair(sRing + rslot * kUnitBytes, &tm_k, ti.h * kDqk + 64 * it,
-                               key0 + static_cast<int>(rank) * kHalfKeys, fbar, pol_kv);
-            else  // V: 64 keys, this CTA's 64 of the 128 value dims
-              tma_load_2d_pair(sRing + rslot * kUnitBytes, &tm_v,
-                               ti.h * kDv + static_cast<int>(rank) * kHalfDv,
-                               key0 + 64 * (it - kKUnits), fbar, pol_kv);
-          }
+        for (int n = 0; n < nblk && ok; ++n, ++blk) {
+          const int slot = blk % kSlots;
+          const uint32_t par = (static_cast<uint32_t>(blk / kSlots) & 1u) ^ 1u;
+          const int key0 = ti.k_start + n * kBlockKeys;
+          // K: this CTA's 64 keys, three 64-dim chunks of the 192
+          if (!(ok = wait(smem_u32(&bars->empty_k[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
+            break;
+          if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full_k[slot]), 2 * kKSlotBytes);
+          const uint32_t kbar = lead(&bars->full_k[slot]);
+#pragma unroll
+          for (int u = 0; u < kKUnits; ++u)
+            tma_load_2d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, &tm_k,
+                             ti.h * kDqk + 64 * u, key0 + static_cast<int>(rank) * kHalfKeys, kbar,
+                             pol_kv);
+          // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
+          if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
+            break;
+          if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full_v[slot]), 2 * kVSlotBytes);
+          const uint32_t vbar = lead(&bars->full_v[slot]);
+#pragma unroll
+          for (int u = 0; u < kVUnits; ++u)
+            tma_load_2d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, &tm_v,
+                             ti.h * kDv + static_cast<int>(rank) * kHalfDv, key0 + 64 * u, vbar,
+                             pol_kv);
         }
       }
       if (!ok && leader) {
         // Unwinding: let the copies already issued land before the CTA exits.
         volatile int no_abort = 0;
-        const int first = max(0, item - kRing);
-        for (int it = first; it < item; ++it)
-          mbar_wait_cluster(smem_u32(&bars->full[it % kRing]),
-                            static_cast<uint32_t>(it / kRing) & 1u, &no_abort, 0, tlim);
+        for (int b = max(0, blk - kSlots); b <= blk; ++b) {
+          const uint32_t par = static_cast<uint32_t>(b / kSlots) & 1u;
+          mbar_wait(smem_u32(&bars->full_k[b % kSlots]), par, &no_abort, 0, tlim / 8);
+          mbar_wait(smem_u32(&bars->full_v[b % kSlots]), par, &no_abort, 0, tlim / 8);
+        }
       }
     }
   } else if (warp == 9) {
@@ -355,20 +370,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return r;
       };
-      auto wait_item = [&](int item) -> bool {
-        return wait_bar(smem_u32(&bars->full[item % kRing]),
-                        static_cast<uint32_t>(item / kRing) & 1u);
+      auto wait_k = [&](int b) -> bool {
+        return wait_bar(smem_u32(&bars->full_k[b % kSlots]), static_cast<uint32_t>(b / kSlots) & 1u);
+      };
+      auto wait_v = [&](int b) -> bool {
+        return wait_bar(smem_u32(&bars->full_v[b % kSlots]), static_cast<uint32_t>(b / kSlots) & 1u);
       };
       auto commit_both = [&](uint64_t* bar) { tc_commit_pair_elect(smem_u32(bar), 0x3); };
-      auto release_item = [&](int item) { commit_both(&bars->empty[item % kRing]); };
       // Descriptors: built once per burst, then advanced by adding to the
       // start-address field (bits 0..13, in 16-byte units); no field carries
       // since every operand lies below 256 KB of shared memory.
-      auto issue_s = [&](int i, int kitem) {
+      auto issue_s = [&](int i, int b) {
+        const uint32_t kslot = sRingK + (b % kSlots) * kKSlotBytes;
 #pragma unroll 1
         for (int c = 0; c < kQkChunks; ++c) {
           uint64_t a = sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes, 16, 1024);
-          uint64_t bd = sdesc_sw128(sRing + ((kitem + c) % kRing) * kUnitBytes, 16, 1024);
+          uint64_t bd = sdesc_sw128(kslot + c * kUnitBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 dims (32 bytes) per MMA
             mma2_ss_elect(tmem + i * 128, a, bd, kIdescQK, (c > 0 || kk > 0) ? 1u : 0u);
@@ -378,11 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         commit_both(&bars->s_full[i]);
       };
-      auto issue_pv = [&](int i, int vitem, bool first) {
+      auto issue_pv = [&](int i, int b, bool first) {
         const uint32_t tO = tmem + 256 + i * 128;
+        const uint32_t vslot = sRingV + (b % kSlots) * kVSlotBytes;
 #pragma unroll 1
         for (int u = 0; u < kVUnits; ++u) {  // 64 keys per unit
-          uint64_t bd = sdesc_sw128(sRing + ((vitem + u) % kRing) * kUnitBytes, kUnitBytes, 1024);
+          uint64_t bd = sdesc_sw128(vslot + u * kUnitBytes, kUnitBytes, 1024);
           uint32_t a_t = tmem + i * 128 + u * 32;  // 16 bf16 of P = 8 columns per MMA
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 keys (16 rows of 128 bytes) per MMA
@@ -393,21 +411,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      int item = 0;           // first ring unit of the current tile
+      int blk = 0;            // first KV block (global count) of the current tile
       int p_cnt[2] = {0, 0};  // P blocks consumed per sub-tile (p_full parity)
       int o_cnt[2] = {0, 0};  // O-using tiles per sub-tile (o_full / o_empty parity)
       // First S MMAs of a tile when the previous tile did not issue them.
-      auto start_tile = [&](const int (&n)[2], int kitem, int k) -> bool {
+      auto start_tile = [&](const int (&n)[2], int b, int k) -> bool {
         for (int i = 0; i < 2; ++i)
           if (!wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k) & 1u)) return false;
         if (max(n[0], n[1]) > 0) {
-          for (int c = 0; c < kKUnits; ++c)
-            if (!wait_item(kitem + c)) return false;
+          if (!wait_k(b)) return false;
           for (int i = 0; i < 2; ++i) {
-            if (n[i] > 0) issue_s(i, kitem);
+            if (n[i] > 0) issue_s(i, b);
             if (n[i] <= 1) commit_both(&bars->q_empty[i]);
           }
-          for (int c = 0; c < kKUnits; ++c) release_item(kitem + c);
+          commit_both(&bars->empty_k[b % kSlots]);
         } else {
           for (int i = 0; i < 2; ++i) commit_both(&bars->q_empty[i]);
         }
@@ -418,27 +435,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileInfo cur = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
       int nb[2];
       tile_blocks(cur, causal, nb);
-      if (cur.valid) ok = start_tile(nb, item, k);
+      if (cur.valid) ok = start_tile(nb, blk, k);
       while (ok && cur.valid) {
         const int nblk = max(nb[0], nb[1]);
         const TileInfo nxt = tile_at(p, k + 1, cluster, nclusters, num_tiles, num_entries);
         int nbn[2];
         tile_blocks(nxt, causal, nbn);
         for (int n = 0; n < nblk && ok; ++n) {
-          const int vitem = item + n * kItemsPerBlock + kKUnits;
+          const int b = blk + n;  // this KV block; the next one is b + 1
           const bool last = n + 1 == nblk;
-          if (!(ok = wait_item(vitem) && wait_item(vitem + 1))) break;
-          // The next KV block is (cur, n+1), or block 0 of the next tile.
-          const int kitem_next = item + (n + 1) * kItemsPerBlock;
+          if (!(ok = wait_v(b))) break;
           bool next_s[2] = {n + 1 < nb[0], n + 1 < nb[1]};
           if (last) {
             next_s[0] = nbn[0] > 0;
             next_s[1] = nbn[1] > 0;
           }
           const bool more = next_s[0] || next_s[1];
-          if (more && !(ok = wait_item(kitem_next) && wait_item(kitem_next + 1) &&
-                             wait_item(kitem_next + 2)))
-            break;
+          if (more && !(ok = wait_k(b + 1))) break;
           for (int i = 0; i < 2 && ok; ++i) {
             if (n < nb[i]) {
               if (n == 0 && !(ok = wait_bar(smem_u32(&bars->o_empty[i]),
@@ -448,21 +461,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   static_cast<uint32_t>(p_cnt[i]) & 1u)))
                 break;
               ++p_cnt[i];
-              issue_pv(i, vitem, n == 0);
+              issue_pv(i, b, n == 0);
               if (n == nb[i] - 1) {
                 commit_both(&bars->o_full[i]);
                 ++o_cnt[i];
               }
             }
-            if (i == 1) {  // both PVs of block n issued: V(n) can be refilled
-              release_item(vitem);
-              release_item(vitem + 1);
-            }
+            if (i == 1) commit_both(&bars->empty_v[b % kSlots]);  // V(b) no longer needed
             if (last && nxt.valid &&
                 !(ok = wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k + 1) & 1u)))
               break;
             if (next_s[i]) {
-              issue_s(i, kitem_next);
+              issue_s(i, b + 1);
               // Q_i is free after the last S MMA of its tile
               const int nbi = last ? nbn[i] : nb[i];
               const int nidx = last ? 0 : n + 1;
@@ -471,12 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               commit_both(&bars->q_empty[i]);  // no S for it in the next tile
             }
           }
-          if (ok && more)
-            for (int c = 0; c < kKUnits; ++c) release_item(kitem_next + c);
+          if (ok && more) commit_both(&bars->empty_k[(b + 1) % kSlots]);  // K(b+1) read by both S
         }
         if (!ok) break;
-        if (nblk == 0 && nxt.valid && !(ok = start_tile(nbn, item, k + 1))) break;
-        item += nblk * kItemsPerBlock;
+        if (nblk == 0 && nxt.valid && !(ok = start_tile(nbn, blk, k + 1))) break;
+        blk += nblk;
         ++k;
         cur = nxt;
         nb[0] = nbn[0];

@@ -40,7 +40,8 @@ WORKLOAD = ("dense varlen causal MLA prefill: 8 sequences, lengths U[512,4096] (
             "fp32 LSE")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
-KERNEL_SRC = os.path.join(ROOT, "mla_prefill_attention_causal_b200", "csrc", "dense_fwd.cuh")
+KERNEL_SRCS = [os.path.join(ROOT, "mla_prefill_attention_causal_b200", "csrc", f)
+               for f in ("dense_fwd.cuh", "ptx.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dense_fwd_varlen16k.md")
 
 
@@ -55,8 +56,13 @@ def load_peaks():
 
 
 def kernel_sha() -> str:
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the dense kernel's sources (the traffic figure is only valid
+    for the source it was measured on)."""
+    h = hashlib.sha256()
+    for path in KERNEL_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic():

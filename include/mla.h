@@ -51,7 +51,8 @@ typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or value  */
   MLA_ERR_UNSUPPORTED = 2, /* not an sm_100 GPU, or an unsupported shape   */
-  MLA_ERR_CUDA = 3         /* a CUDA runtime/driver call or launch failed  */
+  MLA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed  */
+  MLA_ERR_SCRATCH_TOO_SMALL = 4 /* call too large for mla_prefill_fwd_noalloc */
 } mla_status;
 
 /* Bits of the device status word. */
@@ -120,6 +121,39 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
                     float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
                     int batch, int num_heads, int total_q, int total_k, void* workspace,
                     size_t workspace_bytes);
+
+/*
+ * mla_prefill_fwd for callers that cannot allocate device memory.
+ *
+ * (The pages have no counterpart to this entry point; it is a convenience of
+ * this library.)  Some callers have no way to obtain the workspace that
+ * mla_prefill_fwd needs: code that must not call cudaMalloc at all (for
+ * example while other work is being recorded, or inside a runtime that owns
+ * every allocation), or a plain C caller with no allocator of its own.  This
+ * variant takes the same arguments minus the workspace and runs the same
+ * kernels with their work list in a fixed scratch array that is part of the
+ * library itself (MLA_NOALLOC_SCRATCH_BYTES of device memory, reserved on
+ * every GPU that loads the library until the process exits).  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Size limit: mla_prefill_workspace_size(batch, total_q) must not exceed
+ *     MLA_NOALLOC_SCRATCH_BYTES, i.e. ceil(total_q / 512) + batch <= 8160;
+ *     larger calls return MLA_ERR_SCRATCH_TOO_SMALL and launch nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first
+ *     call before capturing work into a graph on that device.
+ *   - All calls share the one array.  The kernels rewrite everything they
+ *     read from it, so nothing needs clearing between calls, but two calls
+ *     whose kernels can overlap on the GPU (different streams without an
+ *     ordering between them) race on it.
+ * Returns the same codes as mla_prefill_fwd, plus MLA_ERR_SCRATCH_TOO_SMALL.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES 65536u
+int mla_prefill_fwd_noalloc(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                            int total_q, int total_k);
 
 /*
  * Merge two partial attention results over disjoint key sets A and B into

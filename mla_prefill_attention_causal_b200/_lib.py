@@ -22,6 +22,8 @@ MLA_OK = 0
 MLA_ERR_INVALID_ARG = 1
 MLA_ERR_UNSUPPORTED = 2
 MLA_ERR_CUDA = 3
+MLA_ERR_SCRATCH_TOO_SMALL = 4
+NOALLOC_SCRATCH_BYTES = 65536
 DEVSTAT_WAIT_TIMEOUT_LOAD = 0x1
 DEVSTAT_WAIT_TIMEOUT_MMA = 0x2
 DEVSTAT_WAIT_TIMEOUT_SOFTMAX = 0x4
@@ -38,6 +40,8 @@ SIGNATURES = {
     "mla_prefill_workspace_size": (_S, [_I, _I]),
     "mla_prefill_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P,
                              _S]),
+    "mla_prefill_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I,
+                                     _I]),
     "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "mla_sparse_prefill_fwd": (_I, [_P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I]),
     "mla_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),

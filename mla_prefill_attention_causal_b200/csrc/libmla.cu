@@ -138,6 +138,30 @@ int encode_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// Scratch for mla_prefill_fwd_noalloc: the dense kernels' work list for
+// callers that cannot allocate.  In host code `g_noalloc_scratch` is only a
+// stand-in symbol; the device address comes from cudaGetSymbolAddress, once
+// per device (with that device current), and is cached here.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(int dev, void** out) {
+  if (g_noalloc_ptr[dev] == nullptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+      }
+      g_noalloc_ptr[dev] = p;
+    }
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
 __global__ void wait_timeout_probe(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -166,6 +190,9 @@ const char* mla_status_string(int status) {
       return "MLA_ERR_UNSUPPORTED: needs an sm_100 (B200) GPU and the supported shapes";
     case MLA_ERR_CUDA:
       return "MLA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MLA_ERR_SCRATCH_TOO_SMALL:
+      return "MLA_ERR_SCRATCH_TOO_SMALL: the call needs more work-list space than the fixed "
+             "scratch of mla_prefill_fwd_noalloc (use mla_prefill_fwd with a workspace)";
     default:
       return "unknown mla_status";
   }
@@ -255,6 +282,25 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
     return MLA_ERR_CUDA;
   }
   return launch_status();
+}
+
+int mla_prefill_fwd_noalloc(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                            int total_q, int total_k) {
+  const size_t need = mla_prefill_workspace_size(batch, total_q);
+  if (need == 0) return MLA_ERR_INVALID_ARG;
+  if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_SCRATCH_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const int st = noalloc_scratch(dev, &scratch);
+  if (st != MLA_OK) return st;
+  return mla_prefill_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                         softmax_scale, causal, out, lse, stream, batch, num_heads, total_q,
+                         total_k, scratch, MLA_NOALLOC_SCRATCH_BYTES);
 }
 
 int mla_attn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

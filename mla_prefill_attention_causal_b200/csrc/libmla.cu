@@ -15,6 +15,7 @@
 #include "mla.h"
 #include "dense_fwd.cuh"
 #include "merge.cuh"
+#include "sparse_fwd.cuh"
 
 namespace {
 
@@ -93,6 +94,10 @@ int prepare_device(int* dev_out) {
       return MLA_ERR_UNSUPPORTED;
     }
   }
+  if (cudaFuncSetAttribute(mla::sparse::sparse_fwd_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           mla::sparse::kSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
   if (encode_fn() == nullptr) return MLA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MLA_ERR_CUDA;
@@ -344,8 +349,33 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* 
   if (topk < 1 || num_tokens < 0 || num_heads < 1 || num_heads > 128 || num_kv_rows < 1)
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
-  (void)stream;
-  return MLA_ERR_UNSUPPORTED;
+  // grid = 2 CTAs per token; TMA row coordinates are int32
+  if (num_tokens > (1 << 30) || static_cast<int64_t>(num_tokens) * num_heads > INT32_MAX)
+    return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  int st = prepare_device(&dev);
+  if (st != MLA_OK) return st;
+  if (num_tokens == 0) return MLA_OK;
+  namespace sp = mla::sparse;
+  CUtensorMap tm_q, tm_kv;
+  if ((st = encode_rows(&tm_q, q, sp::kDl, static_cast<uint64_t>(num_tokens) * num_heads, sp::kM)) !=
+          MLA_OK ||
+      (st = encode_rows(&tm_kv, kv_latent, sp::kDl, static_cast<uint64_t>(num_kv_rows), 1)) != MLA_OK)
+    return st;
+  sp::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.indices = indices;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_tokens = num_tokens;
+  p.num_heads = num_heads;
+  p.num_rows = num_kv_rows;
+  p.topk = topk;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+  p.timeout_ns = wait_timeout_ns();
+  sp::sparse_fwd_kernel<<<2 * num_tokens, sp::kThreads, sp::kSmemBytes,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(tm_q, tm_kv, p);
+  return launch_status();
 }
 
 int mla_device_status(unsigned int* status, int reset) {

@@ -1,0 +1,417 @@
+// Absorbed top-k sparse MLA prefill forward for sm_100a.
+//
+// For token t and head h: O[t,h,:] = sum_r softmax_r(scale * q[t,h,:] .
+// kv[idx[t,r], :]) * kv[idx[t,r], 0:512] over the valid slots r of the
+// token's index list (the "SparseFlashMla" README, Description -- Formula,
+// with K~ = V~ the selected rows; Parameters: -1 marks an invalid slot;
+// Constraints: one index list per token shared by all heads), over the BF16
+// latent cache of the Mojo "mla_prefill_branch_sparse_fp8" absorbed branch
+// (576 = 512 latent + 64 rope dims; V is the first 512).
+//
+// All heads of a token share the selected rows, so the heads are the MMA's
+// M dimension (128 rows; fewer heads are padded).  With 128 heads the
+// output alone (128 x 512 fp32) would fill the whole TMEM, so each token is
+// handled by two CTAs, CTA `half` producing value dims [256 half, +256);
+// both compute the scores.  Per CTA (192 threads):
+//   warps 0-3  softmax + epilogue (thread = head row = TMEM lane); they also
+//              write Q dims [0, 256) into TMEM, the A operand of those MMAs
+//   warp  4    producer: TMA of Q dims [256, 576) into shared memory, and the
+//              key rows, gathered four at a time (tile::gather4) from the
+//              index list, into two chunk slots of 64 keys x 576 dims (72 KB)
+//   warp  5    MMA issuer
+// TMEM (512 columns): S buffers [0,64) and [64,128) (P overwrites their
+// first 32 columns), Q dims 0-255 as bf16 pairs [128,256), O [256,512).
+// MMA order: S(0), S(1), PV(0), S(2), PV(1), ... (S of the next chunk runs
+// while the current chunk's softmax does).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace mla {
+namespace sparse {
+
+constexpr int kM = 128;                          // heads per MMA (rows)
+constexpr int kDl = 576;                         // 512 latent + 64 rope
+constexpr int kDv = 512;
+constexpr int kDvHalf = 256;                     // value dims per CTA
+constexpr int kChunk = 64;                       // keys per chunk (MMA N of S)
+constexpr int kUnits = kDl / 64;                 // 9 units of 64 dims per chunk
+constexpr int kUnitBytes = kChunk * 128;         // 64 keys x 64 bf16 = 8 KB
+constexpr int kSlotBytes = kUnits * kUnitBytes;  // 72 KB
+constexpr int kSlots = 2;
+constexpr int kQtDims = 256;                     // Q dims in TMEM
+constexpr int kQsChunks = (kDl - kQtDims) / 64;  // 5 chunks of 128 rows x 64 dims
+constexpr int kQChunkBytes = kM * 128;           // 16 KB
+constexpr int kQsBytes = kQsChunks * kQChunkBytes;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kColQ = 128;
+constexpr int kColO = 256;
+
+struct alignas(8) Bars {
+  uint64_t q_full;          // TMA bytes of Q's shared-memory part
+  uint64_t qt_ready;        // 4 softmax warps wrote Q's TMEM part
+  uint64_t full[kSlots];    // gathered bytes of a chunk
+  uint64_t empty[kSlots];   // the chunk's PV MMAs done
+  uint64_t s_full[2];
+  uint64_t p_full[2];       // 4 softmax warps
+  uint64_t pv_done;         // one phase per PV(c)
+  uint64_t o_full;
+  uint64_t drain;
+  uint64_t valid_mask[kSlots];  // bit j: key j of the chunk in the slot is a valid row
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr int kSmemBytes = 1024 + kQsBytes + kSlots * kSlotBytes + static_cast<int>(sizeof(Bars));
+static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
+
+struct Params {
+  const __nv_bfloat16* q;  // [T, H, 576]
+  const int* indices;      // [T, topk]
+  __nv_bfloat16* out;      // [T, H, 512]
+  float* lse;              // [H, T] or null
+  int num_tokens;
+  int num_heads;
+  int num_rows;
+  int topk;
+  float scale_log2;
+  uint64_t timeout_ns;
+};
+
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChunk, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kDvHalf, true);
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_kv, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>(blockIdx.x >> 1);
+  const int half = static_cast<int>(blockIdx.x & 1);
+  const int nchunks = (p.topk + kChunk - 1) / kChunk;
+
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sQ = smem_u32(base);
+  const uint32_t sRing = sQ + kQsBytes;
+  Bars* bars = reinterpret_cast<Bars*>(base + kQsBytes + kSlots * kSlotBytes);
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->qt_ready), 4);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_full[i]), 4);
+    }
+    mbar_init(smem_u32(&bars->pv_done), 1);
+    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint64_t tlim = p.timeout_ns;
+  auto warp_wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, tlim));
+  };
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- producer
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_kv);
+      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
+      for (int c = 0; c < kQsChunks; ++c)
+        tma_load_2d_hint(sQ + c * kQChunkBytes, &tm_q, kQtDims + 64 * c, t * p.num_heads,
+                         smem_u32(&bars->q_full), pol_q);
+    }
+    const int* idx_row = p.indices + static_cast<size_t>(t) * p.topk;
+    int issued = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int slot = c % kSlots;
+      if (!warp_wait(smem_u32(&bars->empty[slot]),
+                     (static_cast<uint32_t>(c / kSlots) & 1u) ^ 1u, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD))
+        break;
+      // lane g (< 16) gathers keys 4g..4g+3 of the chunk; invalid slots load
+      // row 0 and are masked by the softmax.
+      int row[4];
+      bool ok4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int key = c * kChunk + 4 * (lane & 15) + j;
+        const int v = key < p.topk ? __ldg(idx_row + key) : -1;
+        ok4[j] = v >= 0 && v < p.num_rows;
+        row[j] = ok4[j] ? v : 0;
+      }
+      uint64_t mask = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t b = __ballot_sync(0xffffffffu, ok4[j]) & 0xFFFFu;  // lanes 0-15
+#pragma unroll
+        for (int g = 0; g < 16; ++g)
+          if (b & (1u << g)) mask |= 1ull << (4 * g + j);
+      }
+      const uint32_t fbar = smem_u32(&bars->full[slot]);
+      if (lane == 0) {
+        bars->valid_mask[slot] = mask;                 // published by the arrive below
+        mbar_arrive_expect_tx(fbar, kSlotBytes);
+      }
+      __syncwarp();
+      if (lane < 16) {
+        const uint32_t dst = sRing + slot * kSlotBytes + lane * 512;  // rows 4g..4g+3
+#pragma unroll 1
+        for (int u = 0; u < kUnits; ++u)
+          tma_gather4(dst + u * kUnitBytes, &tm_kv, 64 * u, row[0], row[1], row[2], row[3], fbar,
+                      pol_kv);
+      }
+      issued = c + 1;
+    }
+    // Do not leave while copies into this CTA's shared memory may be in
+    // flight (only possible after a wait gave up elsewhere).
+    volatile int no_abort = 0;
+    mbar_wait(smem_u32(&bars->q_full), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim);
+    for (int c = issued > kSlots ? issued - kSlots : 0; c < issued; ++c)
+      mbar_wait(smem_u32(&bars->full[c % kSlots]), static_cast<uint32_t>(c / kSlots) & 1u,
+                &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim);
+  } else if (warp == 5) {
+    // -------------------------------------------------------- MMA issuer
+    bool ok = true;
+    auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+      const bool r = warp_wait(bar, parity, MLA_DEVSTAT_WAIT_TIMEOUT_MMA);
+      tc_fence_after();
+      return r;
+    };
+    auto issue_s = [&](int c) {
+      const int buf = c & 1;
+      const uint32_t kv = sRing + (c % kSlots) * kSlotBytes;
+      // dims 0-255: A = Q from TMEM
+#pragma unroll 1
+      for (int u = 0; u < kQtDims / 64; ++u) {
+        uint64_t bd = sdesc_sw128(kv + u * kUnitBytes, 16, 1024);
+        uint32_t a_t = tmem + kColQ + u * 32;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_ts_elect(tmem + buf * kChunk, a_t, bd, kIdescS, (u > 0 || kk > 0) ? 1u : 0u);
+          a_t += 8;
+          bd += 2;
+        }
+      }
+      // dims 256-575: A = Q from shared memory
+#pragma unroll 1
+      for (int u = kQtDims / 64; u < kUnits; ++u) {
+        uint64_t bd = sdesc_sw128(kv + u * kUnitBytes, 16, 1024);
+        uint64_t a = sdesc_sw128(sQ + (u - kQtDims / 64) * kQChunkBytes, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_ss_elect(tmem + buf * kChunk, a, bd, kIdescS, 1u);
+          a += 2;
+          bd += 2;
+        }
+      }
+      tc_commit_elect(smem_u32(&bars->s_full[buf]));
+    };
+    auto issue_pv = [&](int c) {
+      const int buf = c & 1;
+      // this CTA's value dims: units 4*half .. 4*half+3 (four 64-dim atoms, LBO 8 KB)
+      const uint32_t vb = sRing + (c % kSlots) * kSlotBytes + 4 * half * kUnitBytes;
+      uint64_t bd = sdesc_sw128(vb, kUnitBytes, 1024);
+      uint32_t a_t = tmem + buf * kChunk;
+#pragma unroll
+      for (int kk = 0; kk < kChunk / 16; ++kk) {  // 16 keys per MMA
+        mma_ts_elect(tmem + kColO, a_t, bd, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
+        a_t += 8;
+        bd += 128;  // 16 key rows of 128 bytes
+      }
+      tc_commit_elect(smem_u32(&bars->pv_done));
+      tc_commit_elect(smem_u32(&bars->empty[c % kSlots]));
+    };
+    ok = wait_bar(smem_u32(&bars->q_full), 0) && wait_bar(smem_u32(&bars->qt_ready), 0);
+    for (int c = 0; c < 2 && c < nchunks && ok; ++c) {
+      if (!(ok = wait_bar(smem_u32(&bars->full[c]), 0))) break;
+      issue_s(c);
+    }
+    for (int c = 0; c < nchunks && ok; ++c) {
+      if (!(ok = wait_bar(smem_u32(&bars->p_full[c & 1]), static_cast<uint32_t>(c >> 1) & 1u)))
+        break;
+      issue_pv(c);
+      const int n2 = c + 2;
+      if (n2 < nchunks) {
+        if (!(ok = wait_bar(smem_u32(&bars->full[n2 % kSlots]),
+                            static_cast<uint32_t>(n2 / kSlots) & 1u)))
+          break;
+        issue_s(n2);
+      }
+    }
+    tc_commit_elect(smem_u32(&bars->o_full));
+    tc_commit_elect(smem_u32(&bars->drain));
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(smem_u32(&bars->drain), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
+  } else {
+    // ---------------------------------------------- softmax + epilogue
+    const int h = threadIdx.x;  // head row = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const bool row_ok = h < p.num_heads;
+    // Q dims 0-255 of this head as bf16 pairs in TMEM columns [kColQ, +128)
+    {
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          p.q + (static_cast<size_t>(t) * p.num_heads + (row_ok ? h : 0)) * kDl);
+#pragma unroll
+      for (int c = 0; c < kQtDims / 32; ++c) {  // 32 dims = 16 columns per store
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 w = row_ok ? __ldg(qrow + 4 * c + i) : make_uint4(0u, 0u, 0u, 0u);
+          v[4 * i] = w.x;
+          v[4 * i + 1] = w.y;
+          v[4 * i + 2] = w.z;
+          v[4 * i + 3] = w.w;
+        }
+        tmem_st_x16(tmem + lane_off + kColQ + 16 * c, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->qt_ready));
+    }
+    const float sl2 = p.scale_log2;
+    const uint64_t c2 = pack_f32x2(sl2, sl2);
+    const Exp2PolyConsts pk2 = exp2_poly_consts();
+    float m_run = -INFINITY;
+    float l_run = 0.0f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c & 1;
+      const uint32_t tS = tmem + lane_off + buf * kChunk;
+      if (!(ok = warp_wait(smem_u32(&bars->s_full[buf]), static_cast<uint32_t>(c >> 1) & 1u,
+                           MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX)))
+        break;
+      // the chunk's validity mask (published with the gather's barrier)
+      if (!(ok = warp_wait(smem_u32(&bars->full[c % kSlots]),
+                           static_cast<uint32_t>(c / kSlots) & 1u, MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX)))
+        break;
+      const uint64_t vmask = *reinterpret_cast<volatile uint64_t*>(&bars->valid_mask[c % kSlots]);
+      tc_fence_after();
+      uint32_t sraw[64];
+      tmem_ld_x32_wait(tS, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+      tmem_ld_x32_wait(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+      float x[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j)
+        x[j] = ((vmask >> j) & 1ull) ? __uint_as_float(sraw[j]) : -INFINITY;
+      float m4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+      for (int j = 4; j < 60; j += 8)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], x[j + q], x[j + 4 + q]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], x[60 + q]);
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float m_new = fmaxf(m_run, mx * sl2);
+      // Lazy rescaling: keep the old maximum unless the new one exceeds it by 8.
+      const bool need = m_new > m_run + 8.0f;
+      float alpha = 1.0f;
+      if (need) {
+        alpha = ex2_approx(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+      const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if ((j & 7) < 5)
+            pk[j] = softmax_pair_mufu(x[32 * cc + 2 * j], x[32 * cc + 2 * j + 1], c2, negm2,
+                                      acc[j & 3]);
+          else
+            pk[j] = softmax_pair_poly(x[32 * cc + 2 * j], x[32 * cc + 2 * j + 1], c2, negm2, pk2,
+                                      acc[j & 3]);
+        }
+        tmem_st_x16(tS + 16u * cc, pk);
+      }
+      l_run += (sum_f32x2(acc[0]) + sum_f32x2(acc[1])) + (sum_f32x2(acc[2]) + sum_f32x2(acc[3]));
+      // O may only be rescaled once PV(c-1) has finished (PV(c) waits for p_full).
+      if (c > 0) {
+        if (!(ok = warp_wait(smem_u32(&bars->pv_done), static_cast<uint32_t>(c - 1) & 1u,
+                             MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX)))
+          break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+          const uint32_t tO = tmem + lane_off + kColO;
+#pragma unroll 1
+          for (int q = 0; q < kDvHalf / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld_x32_wait(tO + 32u * q, o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st_x32(tO + 32u * q, o);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[buf]));
+    }
+
+    // --------------------------------------------------------- epilogue
+    if (ok && (ok = warp_wait(smem_u32(&bars->o_full), 0, MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX))) {
+      tc_fence_after();
+      const bool seen = m_run != -INFINITY;  // some valid slot
+      const float inv = seen ? 1.0f / l_run : 0.0f;
+      uint4* orow = reinterpret_cast<uint4*>(
+          p.out + (static_cast<size_t>(t) * p.num_heads + h) * kDv + half * kDvHalf);
+      const uint32_t tO = tmem + lane_off + kColO;
+#pragma unroll 1
+      for (int q = 0; q < kDvHalf / 32; ++q) {
+        uint32_t o[32];
+        tmem_ld_x32_wait(tO + 32u * q, o);
+        if (row_ok) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
+                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv);
+            orow[4 * q + v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+      if (row_ok && half == 0 && p.lse != nullptr)
+        p.lse[static_cast<size_t>(h) * p.num_tokens + t] =
+            seen ? (m_run + lg2_approx(l_run)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace sparse
+}  // namespace mla

@@ -1,0 +1,119 @@
+"""GPU parity: absorbed top-k sparse MLA prefill against the fp64 oracle.
+
+The kernel handles a token with two CTAs (value dims 0-255 and 256-511),
+64 selected rows per chunk, 128 heads as the MMA rows.  The cases cover a
+ragged last chunk, fewer heads than 128, -1 padding, out-of-range indices,
+a token with no valid index, duplicates, topk = 1, and the 4096-token
+workload (with and without padding) on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mla_synth as syn
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+from gpu_util import assert_lse_close, assert_out_close, dev_bf16, dev_i32, to_f64  # noqa: E402
+
+
+def run_sparse(case, indices=None, want_lse=True):
+    import mla_prefill_attention_causal_b200 as mla
+    idx = case["indices"] if indices is None else indices
+    out, lse = mla.mla_sparse_prefill_fwd(dev_bf16(case["q"]), dev_bf16(case["kv"]), dev_i32(idx),
+                                          case["scale"], return_lse=want_lse)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def check_sparse(case, indices=None, tokens=None):
+    idx = case["indices"] if indices is None else indices
+    out, lse = run_sparse(case, idx)
+    ref_o, ref_l = oracle.sparse_prefill(case["q"], case["kv"], idx, case["scale"], tokens=tokens)
+    if tokens is None:
+        got_o, got_l = to_f64(out), lse.cpu().numpy().astype(np.float64)
+    else:
+        sel = torch.as_tensor(list(tokens), device=out.device)
+        got_o = to_f64(out.index_select(0, sel))
+        got_l = lse.index_select(1, sel).cpu().numpy().astype(np.float64)
+    assert_out_close(got_o, ref_o, "sparse out")
+    assert_lse_close(got_l, ref_l, "sparse lse")
+    return out, lse
+
+
+def test_small_full_check_ragged_chunk(cuda_ok):
+    # topk 200 = 3 full chunks of 64 + 8; early tokens padded with -1
+    case = syn.sparse_case(num_tokens=9, num_heads=128, num_rows=260, topk=200, first_pos=190,
+                           seed=41)
+    assert (case["indices"] < 0).any()
+    check_sparse(case)
+
+
+@pytest.mark.parametrize("heads", [1, 16, 50, 127])
+def test_fewer_heads_than_mma_rows(cuda_ok, heads):
+    case = syn.sparse_case(num_tokens=6, num_heads=heads, num_rows=500, topk=130, first_pos=400,
+                           seed=42 + heads)
+    check_sparse(case)
+
+
+def test_topk_one_and_single_valid_index(cuda_ok):
+    case = syn.sparse_case(num_tokens=4, num_heads=128, num_rows=64, topk=1, first_pos=10,
+                           seed=43)
+    check_sparse(case)
+    case = syn.sparse_case(num_tokens=4, num_heads=128, num_rows=64, topk=96, first_pos=0,
+                           seed=44)
+    idx = np.full_like(case["indices"], -1)
+    idx[:, 77] = [3, 0, 63, 31]  # one valid slot per token, in the second chunk
+    check_sparse(case, idx)
+
+
+def test_all_padding_and_out_of_range_rows(cuda_ok):
+    case = syn.sparse_case(num_tokens=5, num_heads=128, num_rows=100, topk=128, first_pos=99,
+                           seed=45)
+    idx = case["indices"].copy()
+    idx[0, :] = -1                      # no valid slot: O = 0, LSE = -inf
+    idx[1, ::3] = 100                   # == num_rows: padding
+    idx[2, 5:40] = -7                   # other negatives: padding
+    idx[3, :] = np.iinfo(np.int32).max  # all out of range
+    out, lse = check_sparse(case, idx)
+    assert torch.count_nonzero(out[0]).item() == 0 and torch.count_nonzero(out[3]).item() == 0
+    assert torch.isneginf(lse[:, 0]).all() and torch.isneginf(lse[:, 3]).all()
+
+
+def test_duplicate_indices_count_twice(cuda_ok):
+    case = syn.sparse_case(num_tokens=3, num_heads=64, num_rows=40, topk=192, first_pos=39,
+                           seed=46)
+    g = np.random.Generator(np.random.PCG64(460))
+    idx = g.integers(0, 40, size=(3, 192)).astype(np.int32)  # many repeats
+    check_sparse(case, idx)
+
+
+def test_lse_optional_and_deterministic(cuda_ok):
+    case = syn.sparse_case(num_tokens=8, num_heads=128, num_rows=1000, topk=256, first_pos=900,
+                           seed=47)
+    a, la = run_sparse(case)
+    b, _ = run_sparse(case, want_lse=False)
+    c, lc = run_sparse(case)
+    assert torch.equal(a, b) and torch.equal(a, c) and torch.equal(la, lc)
+
+
+def test_large_values_do_not_overflow(cuda_ok):
+    # q x 32: scores with a standard deviation of 32 (natural-log units) make the
+    # running maximum jump between chunks and the weights nearly one-hot
+    case = syn.sparse_case(num_tokens=3, num_heads=128, num_rows=300, topk=256, first_pos=299,
+                           seed=48)
+    q = case["q"].copy()
+    widened = (q[1].astype(np.uint32) << np.uint32(16)).view(np.float32)
+    q[1] = syn.f32_to_bf16_bits(widened * np.float32(32.0))  # exact: a power of two
+    case = dict(case, q=q)
+    check_sparse(case)
+
+
+@pytest.mark.parametrize("padded", [False, True])
+def test_workload_4096_tokens_sampled(cuda_ok, padded):
+    case = syn.sparse_config(seed=5, padded=padded)
+    g = np.random.Generator(np.random.PCG64(49))
+    tokens = sorted({0, 1, 63, 64, 2046, 2047, 2048, 4095} | set(int(x) for x in
+                                                                   g.integers(0, 4096, size=8)))
+    check_sparse(case, tokens=tokens)

@@ -52,6 +52,20 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity)
 // try_wait that may suspend the thread (without using issue slots) for up to
 // kSuspendHintNs while the phase is incomplete; the hardware resumes it as
 // soon as the phase completes.
+// Non-blocking test of a phase (acquire at CTA scope when it succeeds).
+__device__ __forceinline__ uint32_t mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok;
+}
 constexpr uint32_t kSuspendHintNs = 200000;
 __device__ __forceinline__ uint32_t mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
   uint32_t ok;

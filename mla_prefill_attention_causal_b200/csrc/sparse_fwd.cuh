@@ -12,13 +12,15 @@
 // M dimension (128 rows; fewer heads are padded).  With 128 heads the
 // output alone (128 x 512 fp32) would fill the whole TMEM, so each token is
 // handled by two CTAs, CTA `half` producing value dims [256 half, +256);
-// both compute the scores.  Per CTA (192 threads):
+// both compute the scores.  Per CTA (256 threads):
 //   warps 0-3  softmax + epilogue (thread = head row = TMEM lane); they also
 //              write Q dims [0, 256) into TMEM, the A operand of those MMAs
-//   warp  4    producer: TMA of Q dims [256, 576) into shared memory, and the
-//              key rows, gathered four at a time (tile::gather4) from the
-//              index list, into two chunk slots of 64 keys x 576 dims (72 KB)
-//   warp  5    MMA issuer
+//   warps 4-6  producers: TMA of Q dims [256, 576) into shared memory, and
+//              the key rows, gathered four at a time (tile::gather4) from the
+//              index list, into two chunk slots of 64 keys x 576 dims (72 KB);
+//              one warp alone cannot issue gathers fast enough, so each warp
+//              takes every third 64-dim unit
+//   warp  7    MMA issuer
 // TMEM (512 columns): S buffers [0,64) and [64,128) (P overwrites their
 // first 32 columns), Q dims 0-255 as bf16 pairs [128,256), O [256,512).
 // MMA order: S(0), S(1), PV(0), S(2), PV(1), ... (S of the next chunk runs
@@ -44,7 +46,9 @@ constexpr int kQtDims = 256;                     // Q dims in TMEM
 constexpr int kQsChunks = (kDl - kQtDims) / 64;  // 5 chunks of 128 rows x 64 dims
 constexpr int kQChunkBytes = kM * 128;           // 16 KB
 constexpr int kQsBytes = kQsChunks * kQChunkBytes;
-constexpr int kThreads = 192;
+constexpr int kLoadWarps = 3;                   // gather issue is split over 3 warps
+constexpr int kMmaWarp = 4 + kLoadWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kTmemCols = 512;
 constexpr int kColQ = 128;
 constexpr int kColO = 256;
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -130,11 +134,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, tlim));
   };
 
-  if (warp == 4) {
-    // ---------------------------------------------------------- producer
+  if (warp >= 4 && warp < kMmaWarp) {
+    // --------------------------------------------------------- producers
+    const int pw = warp - 4;
     const uint64_t pol_kv = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
-    if (lane == 0) {
+    if (pw == 0 && lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_kv);
       mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
@@ -149,35 +154,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(smem_u32(&bars->empty[slot]),
                      (static_cast<uint32_t>(c / kSlots) & 1u) ^ 1u, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD))
         break;
-      // lane g (< 16) gathers keys 4g..4g+3 of the chunk; invalid slots load
-      // row 0 and are masked by the softmax.
-      int row[4];
-      bool ok4[4];
+      // Lane g (< 16) gathers keys 4g..4g+3 of the chunk with one tile::gather4
+      // per 64-dim unit.  An invalid slot (padding, out of range, past topk)
+      // is masked by the softmax; its row repeats a valid row of the same
+      // group, so padding neither adds L2 lines nor sends every CTA to one
+      // row.  A group with no valid row is not loaded at all, except on a
+      // slot's first use, where it loads distinct small rows so that the
+      // slot only ever holds finite cache data (masked keys still pass
+      // through the MMAs with zero weight).
+      const int g = lane & 15;
+      int v[4];
+      bool okj[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int key = c * kChunk + 4 * (lane & 15) + j;
-        const int v = key < p.topk ? __ldg(idx_row + key) : -1;
-        ok4[j] = v >= 0 && v < p.num_rows;
-        row[j] = ok4[j] ? v : 0;
+        const int key = c * kChunk + 4 * g + j;
+        v[j] = key < p.topk ? __ldg(idx_row + key) : -1;
+        okj[j] = v[j] >= 0 && v[j] < p.num_rows;
       }
+      const int first = okj[0] ? v[0] : okj[1] ? v[1] : okj[2] ? v[2] : okj[3] ? v[3] : -1;
+      int row[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        row[j] = okj[j] ? v[j] : first >= 0 ? first : (4 * g + j) % p.num_rows;
+      const bool load = first >= 0 || c < kSlots;
+      const uint32_t loads = __ballot_sync(0xffffffffu, load) & 0xFFFFu;
       uint64_t mask = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t b = __ballot_sync(0xffffffffu, ok4[j]) & 0xFFFFu;  // lanes 0-15
+        const uint32_t b = __ballot_sync(0xffffffffu, okj[j]) & 0xFFFFu;  // lanes 0-15
 #pragma unroll
-        for (int g = 0; g < 16; ++g)
-          if (b & (1u << g)) mask |= 1ull << (4 * g + j);
+        for (int q = 0; q < 16; ++q)
+          if (b & (1u << q)) mask |= 1ull << (4 * q + j);
       }
       const uint32_t fbar = smem_u32(&bars->full[slot]);
-      if (lane == 0) {
-        bars->valid_mask[slot] = mask;                 // published by the arrive below
-        mbar_arrive_expect_tx(fbar, kSlotBytes);
+      if (pw == 0 && lane == 0) {
+        bars->valid_mask[slot] = mask;  // published by the arrive below
+        mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(__popc(loads)) * (kUnits * 512u));
       }
       __syncwarp();
-      if (lane < 16) {
+      if (lane < 16 && load) {
         const uint32_t dst = sRing + slot * kSlotBytes + lane * 512;  // rows 4g..4g+3
 #pragma unroll 1
-        for (int u = 0; u < kUnits; ++u)
+        for (int u = pw; u < kUnits; u += kLoadWarps)
           tma_gather4(dst + u * kUnitBytes, &tm_kv, 64 * u, row[0], row[1], row[2], row[3], fbar,
                       pol_kv);
       }
@@ -190,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = issued > kSlots ? issued - kSlots : 0; c < issued; ++c)
       mbar_wait(smem_u32(&bars->full[c % kSlots]), static_cast<uint32_t>(c / kSlots) & 1u,
                 &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim);
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------------------------------- MMA issuer
     bool ok = true;
     auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -243,20 +261,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_elect(smem_u32(&bars->empty[c % kSlots]));
     };
     ok = wait_bar(smem_u32(&bars->q_full), 0) && wait_bar(smem_u32(&bars->qt_ready), 0);
-    for (int c = 0; c < 2 && c < nchunks && ok; ++c) {
-      if (!(ok = wait_bar(smem_u32(&bars->full[c]), 0))) break;
-      issue_s(c);
-    }
-    for (int c = 0; c < nchunks && ok; ++c) {
-      if (!(ok = wait_bar(smem_u32(&bars->p_full[c & 1]), static_cast<uint32_t>(c >> 1) & 1u)))
-        break;
-      issue_pv(c);
-      const int n2 = c + 2;
-      if (n2 < nchunks) {
-        if (!(ok = wait_bar(smem_u32(&bars->full[n2 % kSlots]),
-                            static_cast<uint32_t>(n2 / kSlots) & 1u)))
+    // Issue S(c) and PV(c) in whichever order their inputs arrive: PV(c)
+    // frees chunk c's slot for the next gather, so it must not queue behind
+    // the wait for a later chunk's rows.  S(c) reuses the S/P buffer of
+    // chunk c-2, so it follows PV(c-2) in issue order.
+    auto ready = [&](uint32_t bar, uint32_t parity) -> bool {
+      return __shfl_sync(0xffffffffu, lane == 0 ? mbar_test_wait(bar, parity) : 0u, 0) != 0u;
+    };
+    int s_next = 0, pv_next = 0;
+    uint64_t t_last = globaltimer_ns();
+    while (ok && pv_next < nchunks) {
+      bool progressed = false;
+      if (pv_next < s_next &&
+          ready(smem_u32(&bars->p_full[pv_next & 1]), static_cast<uint32_t>(pv_next >> 1) & 1u)) {
+        if (!(ok = wait_bar(smem_u32(&bars->p_full[pv_next & 1]),
+                            static_cast<uint32_t>(pv_next >> 1) & 1u)))
           break;
-        issue_s(n2);
+        issue_pv(pv_next++);
+        progressed = true;
+      }
+      if (s_next < nchunks && s_next <= pv_next + 1 &&
+          ready(smem_u32(&bars->full[s_next % kSlots]),
+                static_cast<uint32_t>(s_next / kSlots) & 1u)) {
+        if (!(ok = wait_bar(smem_u32(&bars->full[s_next % kSlots]),
+                            static_cast<uint32_t>(s_next / kSlots) & 1u)))
+          break;
+        issue_s(s_next++);
+        progressed = true;
+      }
+      if (progressed) {
+        t_last = globaltimer_ns();
+      } else {
+        if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer_ns() - t_last > tlim) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            atomicOr(&g_mla_status, MLA_DEVSTAT_WAIT_TIMEOUT_MMA);
+          }
+          ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        __nanosleep(32);
       }
     }
     tc_commit_elect(smem_u32(&bars->o_full));
@@ -407,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

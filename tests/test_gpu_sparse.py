@@ -81,6 +81,20 @@ def test_all_padding_and_out_of_range_rows(cuda_ok):
     assert torch.isneginf(lse[:, 0]).all() and torch.isneginf(lse[:, 3]).all()
 
 
+def test_unloaded_groups_and_late_valid_slots(cuda_ok):
+    # Groups of four slots with no valid index are not loaded after a slot's
+    # first use; the chunk then still holds earlier rows of the same token.
+    case = syn.sparse_case(num_tokens=4, num_heads=128, num_rows=5000, topk=320, first_pos=4999,
+                           seed=50)
+    idx = case["indices"].copy()
+    idx[0, :] = -1                       # five chunks, nothing valid
+    idx[1, :300] = -1                    # valid slots only in the last chunk
+    idx[2, 64:256] = -1                  # whole chunks 1-3 padded between valid ones
+    idx[3, 4:320:8] = -1                 # a padded slot in every other group
+    out, lse = check_sparse(case, idx)
+    assert torch.count_nonzero(out[0]).item() == 0 and torch.isneginf(lse[:, 0]).all()
+
+
 def test_duplicate_indices_count_twice(cuda_ok):
     case = syn.sparse_case(num_tokens=3, num_heads=64, num_rows=40, topk=192, first_pos=39,
                            seed=46)

@@ -357,13 +357,13 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* 
   if (st != MLA_OK) return st;
   if (num_tokens == 0) return MLA_OK;
   namespace sp = mla::sparse;
-  CUtensorMap tm_q, tm_kv;
+  CUtensorMap tm_q;
   if ((st = encode_rows(&tm_q, q, sp::kDl, static_cast<uint64_t>(num_tokens) * num_heads, sp::kM)) !=
-          MLA_OK ||
-      (st = encode_rows(&tm_kv, kv_latent, sp::kDl, static_cast<uint64_t>(num_kv_rows), 1)) != MLA_OK)
+      MLA_OK)
     return st;
   sp::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kv = static_cast<const __nv_bfloat16*>(kv_latent);
   p.indices = indices;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -374,7 +374,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* 
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
   p.timeout_ns = wait_timeout_ns();
   sp::sparse_fwd_kernel<<<2 * num_tokens, sp::kThreads, sp::kSmemBytes,
-                          reinterpret_cast<cudaStream_t>(stream)>>>(tm_q, tm_kv, p);
+                          reinterpret_cast<cudaStream_t>(stream)>>>(tm_q, p);
   return launch_status();
 }
 

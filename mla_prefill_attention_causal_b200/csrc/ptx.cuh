@@ -128,6 +128,28 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       "r"(bar), "l"(policy)
       : "memory");
 }
+// ---------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy through the load/store path.  `src_bytes`
+// (0 or 16) bytes are read; the rest of the 16 are zero-filled, so 0 reads
+// nothing and writes zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` (without raising its expected count) once every cp.async
+// this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// Order this thread's view of shared memory (including data it saw land
+// through a barrier) before its later async-proxy operations, such as
+// tcgen05.mma reading shared-memory operands.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

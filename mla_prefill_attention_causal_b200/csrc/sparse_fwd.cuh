@@ -12,15 +12,18 @@
 // M dimension (128 rows; fewer heads are padded).  With 128 heads the
 // output alone (128 x 512 fp32) would fill the whole TMEM, so each token is
 // handled by two CTAs, CTA `half` producing value dims [256 half, +256);
-// both compute the scores.  Per CTA (256 threads):
-//   warps 0-3  softmax + epilogue (thread = head row = TMEM lane); they also
-//              write Q dims [0, 256) into TMEM, the A operand of those MMAs
-//   warps 4-6  producers: TMA of Q dims [256, 576) into shared memory, and
-//              the key rows, gathered four at a time (tile::gather4) from the
-//              index list, into two chunk slots of 64 keys x 576 dims (72 KB);
-//              one warp alone cannot issue gathers fast enough, so each warp
-//              takes every third 64-dim unit
-//   warp  7    MMA issuer
+// both compute the scores.  Per CTA (416 threads):
+//   warps 0-3   softmax + epilogue (thread = head row = TMEM lane); they also
+//               write Q dims [0, 256) into TMEM, the A operand of those MMAs
+//   warps 4-11  loaders: the chunk's key rows (64 keys x 576 dims, 72 KB) are
+//               copied with 16-byte cp.async, eight threads per row, into one
+//               of two chunk slots laid out as the MMAs' 128-byte-swizzled
+//               K-major tiles; padded slots are zero-filled without a read.
+//               (Random 1152-byte rows stream several times faster this way
+//               than through tile::gather4, whose issue rate caps one SM's
+//               gather bandwidth well below what the tensor cores consume.)
+//   warp  12    MMA issuer; also the TMA of Q dims [256, 576) into shared
+//               memory
 // TMEM (512 columns): S buffers [0,64) and [64,128) (P overwrites their
 // first 32 columns), Q dims 0-255 as bf16 pairs [128,256), O [256,512).
 // MMA order: S(0), S(1), PV(0), S(2), PV(1), ... (S of the next chunk runs
@@ -46,7 +49,8 @@ constexpr int kQtDims = 256;                     // Q dims in TMEM
 constexpr int kQsChunks = (kDl - kQtDims) / 64;  // 5 chunks of 128 rows x 64 dims
 constexpr int kQChunkBytes = kM * 128;           // 16 KB
 constexpr int kQsBytes = kQsChunks * kQChunkBytes;
-constexpr int kLoadWarps = 3;                   // gather issue is split over 3 warps
+constexpr int kLoadWarps = 8;
+constexpr int kLoaders = 32 * kLoadWarps;
 constexpr int kMmaWarp = 4 + kLoadWarps;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kTmemCols = 512;
@@ -56,14 +60,13 @@ constexpr int kColO = 256;
 struct alignas(8) Bars {
   uint64_t q_full;          // TMA bytes of Q's shared-memory part
   uint64_t qt_ready;        // 4 softmax warps wrote Q's TMEM part
-  uint64_t full[kSlots];    // gathered bytes of a chunk
+  uint64_t full[kSlots];    // every loader thread's copies of a chunk landed
   uint64_t empty[kSlots];   // the chunk's PV MMAs done
   uint64_t s_full[2];
   uint64_t p_full[2];       // 4 softmax warps
   uint64_t pv_done;         // one phase per PV(c)
   uint64_t o_full;
   uint64_t drain;
-  uint64_t valid_mask[kSlots];  // bit j: key j of the chunk in the slot is a valid row
   uint32_t tmem_base;
   int abort;
 };
@@ -73,6 +76,7 @@ static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory above the per-CTA
 
 struct Params {
   const __nv_bfloat16* q;  // [T, H, 576]
+  const __nv_bfloat16* kv; // [N, 576]
   const int* indices;      // [T, topk]
   __nv_bfloat16* out;      // [T, H, 512]
   float* lse;              // [H, T] or null
@@ -88,8 +92,7 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChunk, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kDvHalf, true);
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_kv, const Params p) {
+    sparse_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&bars->q_full), 1);
     mbar_init(smem_u32(&bars->qt_ready), 4);
     for (int i = 0; i < kSlots; ++i) {
-      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->full[i]), kLoaders);
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -135,79 +138,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp >= 4 && warp < kMmaWarp) {
-    // --------------------------------------------------------- producers
-    const int pw = warp - 4;
-    const uint64_t pol_kv = l2_policy_evict_last();
-    const uint64_t pol_q = l2_policy_evict_first();
-    if (pw == 0 && lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_kv);
-      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
-      for (int c = 0; c < kQsChunks; ++c)
-        tma_load_2d_hint(sQ + c * kQChunkBytes, &tm_q, kQtDims + 64 * c, t * p.num_heads,
-                         smem_u32(&bars->q_full), pol_q);
-    }
+    // ------------------------------------------------------------ loaders
+    // Thread i copies 16-byte column j = i % 8 of every 64-dim unit of keys
+    // i / 8 and i / 8 + 32; in the 128-byte swizzle that column of key k
+    // sits at 16-byte position j ^ (k % 8) of the key's 128-byte row.
+    const int li = threadIdx.x - 128;
+    const int j = li & 7;
+    const int k0 = li >> 3;  // 0..31
     const int* idx_row = p.indices + static_cast<size_t>(t) * p.topk;
-    int issued = 0;
+    auto fetch = [&](int c, int r) -> int {
+      const int key = c * kChunk + k0 + 32 * r;
+      return key < p.topk ? __ldg(idx_row + key) : -1;
+    };
+    int vn0 = fetch(0, 0), vn1 = fetch(0, 1);
     for (int c = 0; c < nchunks; ++c) {
       const int slot = c % kSlots;
+      const int v0 = vn0, v1 = vn1;
+      if (c + 1 < nchunks) {  // next chunk's indices load while this one waits
+        vn0 = fetch(c + 1, 0);
+        vn1 = fetch(c + 1, 1);
+      }
       if (!warp_wait(smem_u32(&bars->empty[slot]),
                      (static_cast<uint32_t>(c / kSlots) & 1u) ^ 1u, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD))
         break;
-      // Lane g (< 16) gathers keys 4g..4g+3 of the chunk with one tile::gather4
-      // per 64-dim unit.  An invalid slot (padding, out of range, past topk)
-      // is masked by the softmax; its row repeats a valid row of the same
-      // group, so padding neither adds L2 lines nor sends every CTA to one
-      // row.  A group with no valid row is not loaded at all, except on a
-      // slot's first use, where it loads distinct small rows so that the
-      // slot only ever holds finite cache data (masked keys still pass
-      // through the MMAs with zero weight).
-      const int g = lane & 15;
-      int v[4];
-      bool okj[4];
+      const uint32_t sbase = sRing + slot * kSlotBytes;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int key = c * kChunk + 4 * g + j;
-        v[j] = key < p.topk ? __ldg(idx_row + key) : -1;
-        okj[j] = v[j] >= 0 && v[j] < p.num_rows;
-      }
-      const int first = okj[0] ? v[0] : okj[1] ? v[1] : okj[2] ? v[2] : okj[3] ? v[3] : -1;
-      int row[4];
+      for (int r = 0; r < 2; ++r) {
+        const int v = r == 0 ? v0 : v1;
+        const int k = k0 + 32 * r;
+        const bool valid = v >= 0 && v < p.num_rows;
+        const __nv_bfloat16* src = p.kv + static_cast<size_t>(valid ? v : 0) * kDl + 8 * j;
+        const uint32_t dst = sbase + k * 128 + ((j ^ (k & 7)) << 4);
+        const uint32_t nbytes = valid ? 16u : 0u;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        row[j] = okj[j] ? v[j] : first >= 0 ? first : (4 * g + j) % p.num_rows;
-      const bool load = first >= 0 || c < kSlots;
-      const uint32_t loads = __ballot_sync(0xffffffffu, load) & 0xFFFFu;
-      uint64_t mask = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t b = __ballot_sync(0xffffffffu, okj[j]) & 0xFFFFu;  // lanes 0-15
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (b & (1u << q)) mask |= 1ull << (4 * q + j);
+        for (int u = 0; u < kUnits; ++u) cp_async_16(dst + u * kUnitBytes, src + 64 * u, nbytes);
       }
-      const uint32_t fbar = smem_u32(&bars->full[slot]);
-      if (pw == 0 && lane == 0) {
-        bars->valid_mask[slot] = mask;  // published by the arrive below
-        mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(__popc(loads)) * (kUnits * 512u));
-      }
-      __syncwarp();
-      if (lane < 16 && load) {
-        const uint32_t dst = sRing + slot * kSlotBytes + lane * 512;  // rows 4g..4g+3
-#pragma unroll 1
-        for (int u = pw; u < kUnits; u += kLoadWarps)
-          tma_gather4(dst + u * kUnitBytes, &tm_kv, 64 * u, row[0], row[1], row[2], row[3], fbar,
-                      pol_kv);
-      }
-      issued = c + 1;
+      cp_async_arrive_noinc(smem_u32(&bars->full[slot]));
     }
-    // Do not leave while copies into this CTA's shared memory may be in
-    // flight (only possible after a wait gave up elsewhere).
-    volatile int no_abort = 0;
-    mbar_wait(smem_u32(&bars->q_full), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim);
-    for (int c = issued > kSlots ? issued - kSlots : 0; c < issued; ++c)
-      mbar_wait(smem_u32(&bars->full[c % kSlots]), static_cast<uint32_t>(c / kSlots) & 1u,
-                &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD, tlim);
+    cp_async_wait_all();  // never leave with copies into shared memory in flight
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------- MMA issuer
     bool ok = true;
@@ -260,6 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_elect(smem_u32(&bars->pv_done));
       tc_commit_elect(smem_u32(&bars->empty[c % kSlots]));
     };
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
+      for (int c = 0; c < kQsChunks; ++c)
+        tma_load_2d_hint(sQ + c * kQChunkBytes, &tm_q, kQtDims + 64 * c, t * p.num_heads,
+                         smem_u32(&bars->q_full), l2_policy_evict_first());
+    }
+    __syncwarp();
     ok = wait_bar(smem_u32(&bars->q_full), 0) && wait_bar(smem_u32(&bars->qt_ready), 0);
     // Issue S(c) and PV(c) in whichever order their inputs arrive: PV(c)
     // frees chunk c's slot for the next gather, so it must not queue behind
@@ -286,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_bar(smem_u32(&bars->full[s_next % kSlots]),
                             static_cast<uint32_t>(s_next / kSlots) & 1u)))
           break;
+        fence_proxy_async_smem();  // the rows landed through the generic proxy
         issue_s(s_next++);
         progressed = true;
       }
@@ -310,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     volatile int no_abort = 0;
     mbar_wait(smem_u32(&bars->drain), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
+    // the Q copy has landed unless a wait gave up before it was seen
+    mbar_wait(smem_u32(&bars->q_full), 0, &no_abort, MLA_DEVSTAT_WAIT_TIMEOUT_MMA, tlim);
   } else {
     // ---------------------------------------------- softmax + epilogue
     const int h = threadIdx.x;  // head row = TMEM lane
@@ -343,17 +322,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
+    const int* idx_row = p.indices + static_cast<size_t>(t) * p.topk;
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1;
       const uint32_t tS = tmem + lane_off + buf * kChunk;
+      // Which of the chunk's 64 slots hold a valid row: each warp reads the
+      // index list itself (two entries per lane); the loads complete while
+      // the warp waits for S.
+      const int key_a = c * kChunk + lane, key_b = key_a + 32;
+      const int ia = key_a < p.topk ? __ldg(idx_row + key_a) : -1;
+      const int ib = key_b < p.topk ? __ldg(idx_row + key_b) : -1;
       if (!(ok = warp_wait(smem_u32(&bars->s_full[buf]), static_cast<uint32_t>(c >> 1) & 1u,
                            MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX)))
         break;
-      // the chunk's validity mask (published with the gather's barrier)
-      if (!(ok = warp_wait(smem_u32(&bars->full[c % kSlots]),
-                           static_cast<uint32_t>(c / kSlots) & 1u, MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX)))
-        break;
-      const uint64_t vmask = *reinterpret_cast<volatile uint64_t*>(&bars->valid_mask[c % kSlots]);
+      const uint64_t vmask =
+          static_cast<uint64_t>(__ballot_sync(0xffffffffu, ia >= 0 && ia < p.num_rows)) |
+          (static_cast<uint64_t>(__ballot_sync(0xffffffffu, ib >= 0 && ib < p.num_rows)) << 32);
       tc_fence_after();
       uint32_t sraw[64];
       tmem_ld_x32_wait(tS, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));

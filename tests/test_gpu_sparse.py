@@ -81,9 +81,9 @@ def test_all_padding_and_out_of_range_rows(cuda_ok):
     assert torch.isneginf(lse[:, 0]).all() and torch.isneginf(lse[:, 3]).all()
 
 
-def test_unloaded_groups_and_late_valid_slots(cuda_ok):
-    # Groups of four slots with no valid index are not loaded after a slot's
-    # first use; the chunk then still holds earlier rows of the same token.
+def test_padded_chunks_and_late_valid_slots(cuda_ok):
+    # Whole chunks of padding (zero-filled, never read from the cache) before
+    # and between valid slots, and padding scattered through every chunk.
     case = syn.sparse_case(num_tokens=4, num_heads=128, num_rows=5000, topk=320, first_pos=4999,
                            seed=50)
     idx = case["indices"].copy()

@@ -8,6 +8,13 @@ causal, fp32 LSE.  Throughput counts causal-adjusted algorithmic FLOPs:
 2 * (192 + 128) * heads * (visible query-key pairs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--workload dense|sparse|sparse-padded]
+
+``--workload sparse`` times the absorbed top-k path instead: one
+``mla_sparse_prefill_fwd`` call over 4096 tokens x 128 heads (q dim 576),
+a 32768-row latent cache and top-k 2048 (``sparse-padded``: the same with
+the tokens at the start of the cache, so early lists carry -1 padding);
+FLOPs count 2 * (576 + 512) * heads per valid slot.
 
 Multi-GPU (torchrun): every rank runs its own independent batch of the
 same workload (weak scaling, no collective on the data path); the value is
@@ -40,9 +47,6 @@ WORKLOAD = ("dense varlen causal MLA prefill: 8 sequences, lengths U[512,4096] (
             "fp32 LSE")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
-KERNEL_SRCS = [os.path.join(ROOT, "mla_prefill_attention_causal_b200", "csrc", f)
-               for f in ("dense_fwd.cuh", "ptx.cuh")]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dense_fwd_varlen16k.md")
 
 
 def load_peaks():
@@ -53,36 +57,6 @@ def load_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
-
-
-def kernel_sha() -> str:
-    """Hash of the dense kernel's sources (the traffic figure is only valid
-    for the source it was measured on)."""
-    h = hashlib.sha256()
-    for path in KERNEL_SRCS:
-        with open(path, "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
-
-
-def recorded_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (otherwise None)."""
-    try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
-        return None
-    vals = {}
-    for line in text.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != kernel_sha():
-        return None
-    try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
 
 
 class ClockSampler:
@@ -149,18 +123,6 @@ def make_workload(seed: int, heads: int = 128):
     return syn.varlen16k_config(seed=seed, num_heads=heads)
 
 
-def oracle_sample(case, heads=(0, 1)):
-    """Time the fp64 oracle on the given heads of the workload (all rows)."""
-    import oracle
-    h = list(heads)
-    t0 = time.perf_counter()
-    oracle.dense_prefill(case["q"][:, h], case["k"][:, h], case["v"][:, h], case["cu_q"],
-                         case["cu_k"], case["scale"], True)
-    dt = time.perf_counter() - t0
-    flops = oracle.dense_flops(case["lens_q"], case["lens_k"], len(h), True)
-    return flops, dt
-
-
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -169,43 +131,340 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def reference_step(case, i: int):
-    """One bounded oracle step: every query row of sequence (i mod B) for
-    head (i mod H), through the fp64 oracle as it stands."""
-    import oracle
-    B, H = len(case["lens_q"]), case["num_heads"]
-    b, h = i % B, i % H
-    q0, q1 = int(case["cu_q"][b]), int(case["cu_q"][b + 1])
-    k0, k1 = int(case["cu_k"][b]), int(case["cu_k"][b + 1])
-    t0 = time.perf_counter()
-    oracle.dense_prefill(case["q"][q0:q1, h:h + 1], case["k"][k0:k1, h:h + 1],
-                         case["v"][k0:k1, h:h + 1], [0, q1 - q0], [0, k1 - k0], case["scale"], True)
-    dt = time.perf_counter() - t0
-    return oracle.dense_flops([q1 - q0], [k1 - k0], 1, True), dt
+def source_sha(files) -> str:
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "mla_prefill_attention_causal_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic_for(profile: str, files):
+    """DRAM bytes per launch recorded in a committed ncu summary, if it was
+    taken on the current source of the kernel (otherwise None)."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != source_sha(files):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# Workloads.  Each builds its seeded inputs (pinned host + device copies),
+# one step of the hot path through the public API, the end-to-end step with
+# host copies, and a bounded oracle sample for the CPU baseline.
+# ---------------------------------------------------------------------------
+
+class DenseWorkload:
+    """Dense varlen causal prefill (the headline metric's configuration)."""
+
+    name = "dense"
+    metric = METRIC
+    kernel = "mla::dense::dense_fwd_kernel"
+    sources = ("dense_fwd.cuh", "ptx.cuh")
+    profile = "dense_fwd_varlen16k.md"
+
+    def __init__(self, dev, seed, heads):
+        import torch
+        import oracle
+        self.case = case = make_workload(seed, heads=heads)
+        self.H = H = case["num_heads"]
+        self.flops = oracle.dense_flops(case["lens_q"], case["lens_k"], H, True)
+        to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+        self.hin = [to_t(case["q"]).pin_memory(), to_t(case["k"]).pin_memory(),
+                    to_t(case["v"]).pin_memory(), torch.from_numpy(case["cu_q"]).pin_memory()]
+        self.q, self.k, self.v, self.cu = [x.to(dev) for x in self.hin]
+        T = self.T = self.q.shape[0]
+        self.out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        self.hout = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory(),
+                     torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.launches = 2  # planner + attention kernel
+
+    def step(self):
+        import mla_prefill_attention_causal_b200 as mla
+        c = self.case
+        mla.mla_prefill_fwd(self.q, self.k, self.v, self.cu, self.cu, c["max_q"], c["max_q"],
+                            c["scale"], causal=True, out=self.out, lse=self.lse)
+
+    def e2e_step(self):
+        for d, h in zip((self.q, self.k, self.v, self.cu), self.hin):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.hout[0].copy_(self.out, non_blocking=True)
+        self.hout[1].copy_(self.lse, non_blocking=True)
+
+    def config(self):
+        c = self.case
+        return {"workload": WORKLOAD, "batch": len(c["lens_q"]), "total_tokens": self.T,
+                "heads": self.H, "seq_lens": c["lens_q"], "flops_per_step": self.flops,
+                "l2": "inputs larger than L2 (Q+K+V %.2f GB > 126 MB); no flush" %
+                      ((self.q.numel() + self.k.numel() + self.v.numel()) * 2 / 1e9)}
+
+    data = "synthetic (seeded N(0,1) bf16, lengths U[512,4096])"
+
+    def oracle_sample(self):
+        """The fp64 oracle on heads 0-5 of the workload (all query rows)."""
+        import oracle
+        c, h = self.case, list(range(6))
+        t0 = time.perf_counter()
+        oracle.dense_prefill(c["q"][:, h], c["k"][:, h], c["v"][:, h], c["cu_q"], c["cu_k"],
+                             c["scale"], True)
+        dt = time.perf_counter() - t0
+        f = oracle.dense_flops(c["lens_q"], c["lens_k"], len(h), True)
+        return f, dt, (f"heads 0-5 of {self.H}, all {self.T} query rows of the same batch "
+                       f"({f:.3e} FLOPs in {dt:.1f} s)")
+
+    def reference_step(self, i):
+        """All query rows of sequence (i mod B) for head (i mod H) through the oracle."""
+        import oracle
+        c = self.case
+        B, H = len(c["lens_q"]), c["num_heads"]
+        b, h = i % B, i % H
+        q0, q1 = int(c["cu_q"][b]), int(c["cu_q"][b + 1])
+        k0, k1 = int(c["cu_k"][b]), int(c["cu_k"][b + 1])
+        t0 = time.perf_counter()
+        oracle.dense_prefill(c["q"][q0:q1, h:h + 1], c["k"][k0:k1, h:h + 1],
+                             c["v"][k0:k1, h:h + 1], [0, q1 - q0], [0, k1 - k0], c["scale"], True)
+        return oracle.dense_flops([q1 - q0], [k1 - k0], 1, True), time.perf_counter() - t0
+
+    reference_sample = "step i = all query rows of sequence (i mod 8) for head (i mod 128)"
+
+
+class SparseWorkload:
+    """Absorbed top-k sparse prefill: 4096 tokens x 128 heads, 32768-row latent
+    cache, top-k 2048 (``padded``: the tokens sit at cache positions 0..4095,
+    so the first 2047 lists carry -1 padding)."""
+
+    metric = ("MLA absorbed sparse prefill attn TFLOPS (valid top-k slots) and % of B200 dense "
+              "BF16 peak, 1 GPU")
+    kernel = "mla::sparse::sparse_fwd_kernel"
+    sources = ("sparse_fwd.cuh", "ptx.cuh")
+    profile = "sparse_fwd_4k.md"
+    data = "synthetic (seeded N(0,1) bf16 q and latent cache, causal top-k index lists)"
+    reference_sample = "step i = all 128 heads of token (i * 997 mod 4096)"
+
+    def __init__(self, dev, seed, heads, padded=False):
+        import torch
+        import mla_synth as syn
+        import oracle
+        self.name = "sparse-padded" if padded else "sparse"
+        self.padded = padded
+        self.case = case = syn.sparse_config(seed=seed, padded=padded)
+        self.H = H = case["num_heads"]
+        self.flops = oracle.sparse_flops(case["indices"], case["num_rows"], H)
+        to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+        self.hin = [to_t(case["q"]).pin_memory(), to_t(case["kv"]).pin_memory(),
+                    torch.from_numpy(case["indices"]).pin_memory()]
+        self.q, self.kv, self.idx = [x.to(dev) for x in self.hin]
+        T = self.T = self.q.shape[0]
+        self.out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        self.hout = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory(),
+                     torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.launches = 1
+
+    def step(self):
+        import mla_prefill_attention_causal_b200 as mla
+        mla.mla_sparse_prefill_fwd(self.q, self.kv, self.idx, self.case["scale"], out=self.out,
+                                   lse=self.lse)
+
+    def e2e_step(self):
+        for d, h in zip((self.q, self.kv, self.idx), self.hin):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.hout[0].copy_(self.out, non_blocking=True)
+        self.hout[1].copy_(self.lse, non_blocking=True)
+
+    def config(self):
+        c = self.case
+        return {"workload": ("absorbed sparse MLA prefill: %d tokens x %d heads, q/latent dim 576 "
+                             "(V = first 512), %d-row latent cache, top-k %d without replacement "
+                             "from the causally visible rows%s, scale 1/sqrt(576), fp32 LSE" %
+                             (self.T, self.H, c["num_rows"], c["topk"],
+                              " (tokens at positions 0..4095: -1 padding)" if self.padded
+                              else " (tokens at the last 4096 positions)")),
+                "tokens": self.T, "heads": self.H, "topk": c["topk"], "cache_rows": c["num_rows"],
+                "flops_per_step": self.flops,
+                "l2": "q + out %.2f GB > 126 MB (the 38 MB cache stays L2-resident); no flush" %
+                      ((self.q.numel() + self.out.numel()) * 2 / 1e9)}
+
+    def _oracle_tokens(self, tokens):
+        import oracle
+        c = self.case
+        t0 = time.perf_counter()
+        oracle.sparse_prefill(c["q"], c["kv"], c["indices"], c["scale"], tokens=tokens)
+        dt = time.perf_counter() - t0
+        f = oracle.sparse_flops(c["indices"][tokens], c["num_rows"], self.H)
+        return f, dt
+
+    def oracle_sample(self):
+        tokens = [int(x) for x in (np.arange(64) * 61) % self.T]
+        f, dt = self._oracle_tokens(tokens)
+        return f, dt, (f"64 of the {self.T} tokens (all heads; tokens 61*i mod {self.T}); "
+                       f"{f:.3e} FLOPs in {dt:.1f} s")
+
+    def reference_step(self, i):
+        return self._oracle_tokens([(i * 997) % self.T])
+
+
+class ChunkedWorkload:
+    """Chunked prefill with context: 4 sequences, each a 2048-token query
+    chunk attending non-causally to a 16384-token prefix and causally to
+    itself, the two partial results combined by ``mla_attn_merge``."""
+
+    name = "chunked"
+    metric = ("MLA chunked prefill (prefix pass + causal self pass + LSE merge) attn TFLOPS "
+              "(causal-adj) and % of B200 dense BF16 peak, 1 GPU")
+    kernel = "mla::dense::dense_fwd_kernel"
+    sources = ("dense_fwd.cuh", "ptx.cuh")
+    profile = "dense_fwd_varlen16k.md"
+    merge_sources = ("merge.cuh",)
+    merge_profile = "merge_chunked.md"
+    data = "synthetic (seeded N(0,1) bf16 query chunks, prefix and self K/V)"
+    reference_sample = ("step i = head (i mod 128) of sequence (i mod 4): prefix pass, self pass "
+                        "and merge of that head's 2048 query rows")
+
+    def __init__(self, dev, seed, heads):
+        import torch
+        import mla_synth as syn
+        import oracle
+        self.case = c = syn.chunked_config(seed=seed, num_heads=heads)
+        self.H = H = c["num_heads"]
+        B, L, P = c["batch"], c["chunk"], c["prefix"]
+        self.flops = (oracle.dense_flops([L] * B, [P] * B, H, False) +
+                      oracle.dense_flops([L] * B, [L] * B, H, True))
+        to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+        self.hin = [to_t(c[k]).pin_memory() for k in ("q", "k_prefix", "v_prefix", "k_self",
+                                                      "v_self")]
+        self.hin += [torch.from_numpy(c["cu_q"]).pin_memory(),
+                     torch.from_numpy(c["cu_prefix"]).pin_memory()]
+        (self.q, self.kp, self.vp, self.ks, self.vs, self.cu_q, self.cu_p) = [
+            x.to(dev) for x in self.hin]
+        T = self.T = self.q.shape[0]
+        mk = lambda: (torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev),
+                      torch.empty((H, T), dtype=torch.float32, device=dev))
+        (self.op, self.lp), (self.os, self.ls), (self.out, self.lse) = mk(), mk(), mk()
+        self.hout = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory(),
+                     torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.launches = 5  # 2 x (planner + attention) + merge
+        self.merge_bytes = 3 * self.out.numel() * 2 + 3 * self.lse.numel() * 4
+        self.merge_events = None
+
+    def step(self):
+        import torch
+        import mla_prefill_attention_causal_b200 as mla
+        c = self.case
+        mla.mla_prefill_fwd(self.q, self.kp, self.vp, self.cu_q, self.cu_p, c["chunk"], c["prefix"],
+                            c["scale"], causal=False, out=self.op, lse=self.lp)
+        mla.mla_prefill_fwd(self.q, self.ks, self.vs, self.cu_q, self.cu_q, c["chunk"], c["chunk"],
+                            c["scale"], causal=True, out=self.os, lse=self.ls)
+        if self.merge_events is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mla.mla_attn_merge(self.op, self.lp, self.os, self.ls, out=self.out, lse_out=self.lse)
+            e1.record()
+            self.merge_events.append((e0, e1))
+        else:
+            mla.mla_attn_merge(self.op, self.lp, self.os, self.ls, out=self.out, lse_out=self.lse)
+
+    def e2e_step(self):
+        for d, h in zip((self.q, self.kp, self.vp, self.ks, self.vs, self.cu_q, self.cu_p),
+                        self.hin):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.hout[0].copy_(self.out, non_blocking=True)
+        self.hout[1].copy_(self.lse, non_blocking=True)
+
+    def config(self):
+        c = self.case
+        return {"workload": ("chunked MLA prefill with context: %d sequences, %d-token query "
+                             "chunks, non-causal prefix of %d tokens plus causal self pass, "
+                             "merged with mla_attn_merge; %d heads, qk 192 / v 128, bf16 N(0,1), "
+                             "scale 1/sqrt(192)" % (c["batch"], c["chunk"], c["prefix"], self.H)),
+                "tokens": self.T, "heads": self.H, "flops_per_step": self.flops,
+                "merge_bytes_per_step": self.merge_bytes,
+                "l2": "prefix K/V %.2f GB > 126 MB; no flush" %
+                      ((self.kp.numel() + self.vp.numel()) * 2 / 1e9)}
+
+    def _oracle_head(self, b, h):
+        import oracle
+        c = self.case
+        L, P = c["chunk"], c["prefix"]
+        sl = lambda a, n, lo: a[lo * n:(lo + 1) * n, h:h + 1]
+        t0 = time.perf_counter()
+        o1, l1 = oracle.dense_prefill(sl(c["q"], L, b), sl(c["k_prefix"], P, b),
+                                      sl(c["v_prefix"], P, b), [0, L], [0, P], c["scale"], False)
+        o2, l2 = oracle.dense_prefill(sl(c["q"], L, b), sl(c["k_self"], L, b),
+                                      sl(c["v_self"], L, b), [0, L], [0, L], c["scale"], True)
+        oracle.attn_merge(o1, l1, o2, l2)
+        dt = time.perf_counter() - t0
+        f = oracle.dense_flops([L], [P], 1, False) + oracle.dense_flops([L], [L], 1, True)
+        return f, dt
+
+    def oracle_sample(self):
+        f, dt = self._oracle_head(0, 0)
+        return f, dt, (f"head 0 of sequence 0 (prefix pass, self pass and merge of its "
+                       f"{self.case['chunk']} query rows): {f:.3e} FLOPs in {dt:.1f} s")
+
+    def reference_step(self, i):
+        return self._oracle_head(i % self.case["batch"], i % self.H)
+
+
+def make(args, dev, rank, world):
+    seed_off = 0 if world == 1 else 1000 * rank
+    if args.workload == "dense":
+        return DenseWorkload(dev, 2 + seed_off, args.heads)
+    if args.workload == "chunked":
+        return ChunkedWorkload(dev, 4 + seed_off, args.heads)
+    return SparseWorkload(dev, 5 + seed_off, args.heads, padded=args.workload == "sparse-padded")
 
 
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
-    import oracle
-    case = make_workload(2)
-    total_flops = oracle.dense_flops(case["lens_q"], case["lens_k"], case["num_heads"], True)
+    # The reference arm runs the oracle on the host only: build the host-side case.
+    if args.workload == "dense":
+        w = DenseWorkload.__new__(DenseWorkload)
+        w.case = make_workload(2)
+        w.H = w.case["num_heads"]
+    elif args.workload == "chunked":
+        import mla_synth as syn
+        w = ChunkedWorkload.__new__(ChunkedWorkload)
+        w.case = syn.chunked_config(seed=4)
+        w.H = w.case["num_heads"]
+    else:
+        import mla_synth as syn
+        w = SparseWorkload.__new__(SparseWorkload)
+        w.padded = args.workload == "sparse-padded"
+        w.case = syn.sparse_config(seed=5, padded=w.padded)
+        w.H, w.T = w.case["num_heads"], w.case["q"].shape[0]
     for i in range(args.warmup):
-        reference_step(case, i)
+        w.reference_step(i)
     flops, secs = 0, 0.0
     for i in range(args.steps):
-        f, dt = reference_step(case, i)
+        f, dt = w.reference_step(i)
         flops += f
         secs += dt
     value = flops / secs / 1e12
-    sample = (f"step i = all query rows of sequence (i mod 8) for head (i mod 128); "
-              f"{args.steps} steps = {flops:.3e} of the workload's {total_flops:.3e} FLOPs")
+    sample = f"{w.reference_sample}; {args.steps} steps = {flops:.3e} FLOPs"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": w.metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": WORKLOAD, "sample": sample},
+        "config": {"workload": WORKLOAD if args.workload == "dense" else args.workload,
+                   "sample": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -219,30 +478,14 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     import torch.distributed as dist
 
     import mla_prefill_attention_causal_b200 as mla
-    import oracle
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    case = make_workload(2 if world == 1 else 2 + 1000 * rank, heads=args.heads)
-    H = case["num_heads"]
-    flops = oracle.dense_flops(case["lens_q"], case["lens_k"], H, True)
-    to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
-    hq, hk, hv = to_t(case["q"]).pin_memory(), to_t(case["k"]).pin_memory(), to_t(case["v"]).pin_memory()
-    hcu = torch.from_numpy(case["cu_q"]).pin_memory()
-    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
-    cu = hcu.to(dev)
-    T = q.shape[0]
-    out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
-    max_q = case["max_q"]
+    w = make(args, dev, rank, world)
     stream = torch.cuda.current_stream()
 
-    def step():
-        mla.mla_prefill_fwd(q, k, v, cu, cu, max_q, max_q, case["scale"], causal=True,
-                            out=out, lse=lse)
-
     for _ in range(max(args.warmup, 3)):
-        step()
+        w.step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -253,93 +496,96 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if hasattr(w, "merge_events"):
+        w.merge_events = []
     ev0.record(stream)
     for _ in range(args.steps):
-        step()
+        w.step()
     ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
+    merge_ms = None
+    if getattr(w, "merge_events", None):
+        merge_ms = sum(a.elapsed_time(b) for a, b in w.merge_events) / len(w.merge_events)
+        w.merge_events = None
     ms_total = ev0.elapsed_time(ev1)
     t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = w.flops * world / (ms_step * 1e-3) / 1e12
     status = mla.mla_device_status(reset=True)
     if args.kernel_only:
         if rank == 0:
-            print(json.dumps({"kernel_only": True, "heads": H, "ms_per_step": ms_step,
-                              "tflops": flops / (ms_step * 1e-3) / 1e12, "device_status": status}),
-                  flush=True)
+            print(json.dumps({"kernel_only": True, "workload": w.name, "heads": w.H,
+                              "ms_per_step": ms_step,
+                              "tflops": w.flops / (ms_step * 1e-3) / 1e12,
+                              "device_status": status}), flush=True)
         return 0
 
     # End to end through the public call with host buffers: H2D of the step's
-    # inputs from pinned memory, the kernel, D2H of out and lse.
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    # inputs from pinned memory, the kernel(s), D2H of out and lse.
     e2e_steps = max(3, min(args.steps, 20))
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        cu.copy_(hcu, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
-
-    e2e_step()
+    w.e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     ev0.record(stream)
     for _ in range(e2e_steps):
-        e2e_step()
+        w.e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
     te = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_ms = float(te.item())
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hcu))
-    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+    h2d = sum(x.numel() * x.element_size() for x in w.hin)
+    d2h = sum(x.numel() * x.element_size() for x in w.hout)
 
     if rank != 0:
         return 0
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = flops / (ms_step * 1e-3) / 1e12  # one kernel launch per step
+    attn_ms = ms_step - (merge_ms or 0.0)  # the attention launches of the step
+    achieved = w.flops / (attn_ms * 1e-3) / 1e12
+    config = w.config()
+    config["parallelism"] = f"replicas x{world} (independent batches)"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": w.metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, lengths U[512,4096])",
-        "config": {"workload": WORKLOAD, "batch": len(case["lens_q"]), "total_tokens": T,
-                   "heads": H, "seq_lens": case["lens_q"], "flops_per_step": flops,
-                   "l2": "inputs larger than L2 (Q+K+V %.2f GB > 126 MB); no flush" %
-                         ((q.numel() + k.numel() + v.numel()) * 2 / 1e9),
-                   "parallelism": f"replicas x{world} (independent batches)"},
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": w.data,
+        "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained",
                                                                      peak)),
-                     "traffic": recorded_traffic(),
-                     "kernel": "mla::dense::dense_fwd_kernel"},
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                     "traffic": recorded_traffic_for(w.profile, w.sources),
+                     "kernel": w.kernel,
+                     "timed": "one public call per step; CUDA events on its stream"},
+        "e2e": {"value": w.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * w.launches,
         "clocks": clocks,
         "device_status": status,
     }
+    if merge_ms is not None:
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        gbs = w.merge_bytes / (merge_ms * 1e-3) / 1e9
+        line["roofline"]["timed"] = ("attention launches of the step (step time minus the "
+                                     "separately event-timed merge)")
+        line["merge_roofline"] = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                  "frac": gbs / hbm, "ms": merge_ms,
+                                  "peak_source": f"{peak_src} hbm_gbs",
+                                  "traffic": recorded_traffic_for(w.merge_profile,
+                                                                  w.merge_sources),
+                                  "kernel": "mla::merge::merge_kernel"}
     if world == 1 and not args.no_cpu_baseline:
-        f, dt = oracle_sample(case, heads=tuple(range(6)))
-        line["cpu_baseline"] = {
-            "value": f / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"heads 0-5 of 128, all {T} query rows of the same batch "
-                      f"({f:.3e} FLOPs in {dt:.1f} s)"}
+        f, dt, sample = w.oracle_sample()
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -354,7 +600,10 @@ def main():
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the kernel only (no e2e, clocks or CPU baseline); for profiling")
     ap.add_argument("--heads", type=int, default=128,
-                    help="heads of the workload (128 for the bench line; fewer for profiling)")
+                    help="heads of the dense workload (128 for the bench line; fewer for profiling)")
+    ap.add_argument("--workload", default="dense", choices=["dense", "chunked", "sparse", "sparse-padded"],
+                    help="dense: the headline configuration; chunked: prefix + self passes and "
+                         "the LSE merge; sparse: the absorbed top-k path")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

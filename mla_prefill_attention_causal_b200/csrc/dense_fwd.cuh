@@ -384,14 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kslot = sRingK + (b % kSlots) * kKSlotBytes;
 #pragma unroll 1
         for (int c = 0; c < kQkChunks; ++c) {
-          uint64_t a = sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes, 16, 1024);
-          uint64_t bd = sdesc_sw128(kslot + c * kUnitBytes, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // 16 dims (32 bytes) per MMA
-            mma2_ss_elect(tmem + i * 128, a, bd, kIdescQK, (c > 0 || kk > 0) ? 1u : 0u);
-            a += 2;
-            bd += 2;
-          }
+          // four MMAs of 16 dims (32 bytes) each
+          mma2_ss_x4_elect(tmem + i * 128, sdesc_sw128(sQ + (i * kQkChunks + c) * kQChunkBytes, 16, 1024),
+                           sdesc_sw128(kslot + c * kUnitBytes, 16, 1024), kIdescQK, c > 0 ? 1u : 0u);
         }
         commit_both(&bars->s_full[i]);
       };
@@ -400,14 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vslot = sRingV + (b % kSlots) * kVSlotBytes;
 #pragma unroll 1
         for (int u = 0; u < kVUnits; ++u) {  // 64 keys per unit
-          uint64_t bd = sdesc_sw128(vslot + u * kUnitBytes, kUnitBytes, 1024);
-          uint32_t a_t = tmem + i * 128 + u * 32;  // 16 bf16 of P = 8 columns per MMA
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // 16 keys (16 rows of 128 bytes) per MMA
-            mma2_ts_elect(tO, a_t, bd, kIdescPV, (!first || u > 0 || kk > 0) ? 1u : 0u);
-            a_t += 8;
-            bd += 128;
-          }
+          // four MMAs of 16 keys (16 rows of 128 bytes; 16 bf16 of P = 8 columns) each
+          mma2_ts_x4_elect(tO, tmem + i * 128 + u * 32,
+                           sdesc_sw128(vslot + u * kUnitBytes, kUnitBytes, 1024), kIdescPV,
+                           (!first || u > 0) ? 1u : 0u);
         }
       };
 

@@ -384,6 +384,115 @@ __device__ __forceinline__ void mma2_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Four consecutive K-steps of M=256 MMAs under one elect: the elected lane
+// issues them back to back, advancing the descriptors' start addresses by
+// `a_step` / `b_step` (16-byte units) between steps.  The first MMA
+// accumulates only if `accumulate` is set; the other three always do.
+__device__ __forceinline__ void mma2_ss_x4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p, e, t;\n"
+      ".reg .b64 a1, a2, a3, b1, b2, b3;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "setp.eq.b32 t, %4, %4;\n"
+      "add.s64 a1, %1, 2;\n"
+      "add.s64 a2, %1, 4;\n"
+      "add.s64 a3, %1, 6;\n"
+      "add.s64 b1, %2, 2;\n"
+      "add.s64 b2, %2, 4;\n"
+      "add.s64 b3, %2, 6;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], a1, b1, %3, t;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], a2, b2, %3, t;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], a3, b3, %3, t;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same with A in TMEM (8 columns per K-step) and B advancing by 128
+// (16 rows of 128 bytes).
+__device__ __forceinline__ void mma2_ts_x4_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p, e, t;\n"
+      ".reg .b32 a1, a2, a3;\n"
+      ".reg .b64 b1, b2, b3;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "setp.eq.b32 t, %4, %4;\n"
+      "add.u32 a1, %1, 8;\n"
+      "add.u32 a2, %1, 16;\n"
+      "add.u32 a3, %1, 24;\n"
+      "add.s64 b1, %2, 128;\n"
+      "add.s64 b2, %2, 256;\n"
+      "add.s64 b3, %2, 384;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [a1], b1, %3, t;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [a2], b2, %3, t;\n"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [a3], b3, %3, t;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Four consecutive K-steps of single-CTA MMAs under one elect: the elected lane
+// issues them back to back, advancing the descriptors' start addresses by
+// `a_step` / `b_step` (16-byte units) between steps.  The first MMA
+// accumulates only if `accumulate` is set; the other three always do.
+__device__ __forceinline__ void mma_ss_x4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p, e, t;\n"
+      ".reg .b64 a1, a2, a3, b1, b2, b3;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "setp.eq.b32 t, %4, %4;\n"
+      "add.s64 a1, %1, 2;\n"
+      "add.s64 a2, %1, 4;\n"
+      "add.s64 a3, %1, 6;\n"
+      "add.s64 b1, %2, 2;\n"
+      "add.s64 b2, %2, 4;\n"
+      "add.s64 b3, %2, 6;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same with A in TMEM (8 columns per K-step) and B advancing by BSTEP
+// (16-byte units): 2 for a K-major B (32 bytes of K), 128 for an MN-major B
+// (16 rows of 128 bytes).
+template <int BSTEP>
+__device__ __forceinline__ void mma_ts_x4_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p, e, t;\n"
+      ".reg .b32 a1, a2, a3;\n"
+      ".reg .b64 b1, b2, b3;\n"
+      "elect.sync _|e, 0xffffffff;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "setp.eq.b32 t, %4, %4;\n"
+      "add.u32 a1, %1, 8;\n"
+      "add.u32 a2, %1, 16;\n"
+      "add.u32 a3, %1, 24;\n"
+      "add.s64 b1, %2, %5;\n"
+      "add.s64 b2, %2, %6;\n"
+      "add.s64 b3, %2, %7;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(BSTEP), "n"(2 * BSTEP),
+      "n"(3 * BSTEP)
+      : "memory");
+}
 // Arrive on the mbarrier at `bar` (same offset) in every CTA of `mask` once
 // all prior tcgen05 operations of this thread have completed.
 __device__ __forceinline__ void tc_commit_pair_elect(uint32_t bar, uint16_t mask) {

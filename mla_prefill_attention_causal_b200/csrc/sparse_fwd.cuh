@@ -190,26 +190,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dims 0-255: A = Q from TMEM
 #pragma unroll 1
       for (int u = 0; u < kQtDims / 64; ++u) {
-        uint64_t bd = sdesc_sw128(kv + u * kUnitBytes, 16, 1024);
-        uint32_t a_t = tmem + kColQ + u * 32;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_ts_elect(tmem + buf * kChunk, a_t, bd, kIdescS, (u > 0 || kk > 0) ? 1u : 0u);
-          a_t += 8;
-          bd += 2;
-        }
+        mma_ts_x4_elect<2>(tmem + buf * kChunk, tmem + kColQ + u * 32,
+                           sdesc_sw128(kv + u * kUnitBytes, 16, 1024), kIdescS, u > 0 ? 1u : 0u);
       }
       // dims 256-575: A = Q from shared memory
 #pragma unroll 1
       for (int u = kQtDims / 64; u < kUnits; ++u) {
-        uint64_t bd = sdesc_sw128(kv + u * kUnitBytes, 16, 1024);
-        uint64_t a = sdesc_sw128(sQ + (u - kQtDims / 64) * kQChunkBytes, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_ss_elect(tmem + buf * kChunk, a, bd, kIdescS, 1u);
-          a += 2;
-          bd += 2;
-        }
+        mma_ss_x4_elect(tmem + buf * kChunk, sdesc_sw128(sQ + (u - kQtDims / 64) * kQChunkBytes, 16, 1024),
+                        sdesc_sw128(kv + u * kUnitBytes, 16, 1024), kIdescS, 1u);
       }
       tc_commit_elect(smem_u32(&bars->s_full[buf]));
     };
@@ -217,14 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = c & 1;
       // this CTA's value dims: units 4*half .. 4*half+3 (four 64-dim atoms, LBO 8 KB)
       const uint32_t vb = sRing + (c % kSlots) * kSlotBytes + 4 * half * kUnitBytes;
-      uint64_t bd = sdesc_sw128(vb, kUnitBytes, 1024);
-      uint32_t a_t = tmem + buf * kChunk;
-#pragma unroll
-      for (int kk = 0; kk < kChunk / 16; ++kk) {  // 16 keys per MMA
-        mma_ts_elect(tmem + kColO, a_t, bd, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
-        a_t += 8;
-        bd += 128;  // 16 key rows of 128 bytes
-      }
+      // four MMAs of 16 keys (16 key rows of 128 bytes) each
+      mma_ts_x4_elect<128>(tmem + kColO, tmem + buf * kChunk, sdesc_sw128(vb, kUnitBytes, 1024),
+                           kIdescPV, c > 0 ? 1u : 0u);
       tc_commit_elect(smem_u32(&bars->pv_done));
       tc_commit_elect(smem_u32(&bars->empty[c % kSlots]));
     };

@@ -168,13 +168,45 @@ __global__ void __launch_bounds__(kPlanThreads)
     for (int mb = 0; mb < nmb; ++mb) atomicAdd(&bins[work_of(Lq, Lk, mb)], 1);
   }
   __syncthreads();
-  if (tid == 0) {  // exclusive prefix over bins in descending work order
-    int run = 0;
-    for (int w = kPlanBins - 1; w >= 0; --w) {
-      const int c = bins[w];
-      bins[w] = run;
-      run += c;
+  {
+    // Exclusive prefix over the bins in descending work order, 4 bins a
+    // thread: warp scans of the thread sums, then a scan of the warp sums.
+    static_assert(kPlanBins == 4 * kPlanThreads, "4 bins per planner thread");
+    __shared__ int warp_sums[kPlanThreads / 32];
+    const int lane = tid & 31, wid = tid >> 5;
+    int c[4], tsum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      c[i] = bins[kPlanBins - 1 - (4 * tid + i)];
+      tsum += c[i];
     }
+    int incl = tsum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      const int w = warp_sums[lane];
+      int wi = w;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, wi, off);
+        if (lane >= off) wi += v;
+      }
+      warp_sums[lane] = wi - w;
+    }
+    __syncthreads();
+    int run = warp_sums[wid] + incl - tsum;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      bins[kPlanBins - 1 - (4 * tid + i)] = run;
+      run += c[i];
+    }
+  }
+  if (tid == 0) {
     // More entries than the workspace holds means cu_seqlens_q does not end
     // at total_q: report it and compute only what fits.
     if (s_total > capacity) atomicOr(&g_mla_status, MLA_DEVSTAT_PLAN_OVERFLOW);

@@ -421,13 +421,34 @@ class ChunkedWorkload:
         return self._oracle_head(i % self.case["batch"], i % self.H)
 
 
+def rank_seed(base: int, rank: int, world: int) -> int:
+    """Seed of a rank's batch: the workload's own seed on one GPU, and a
+    distinct batch per rank under weak scaling."""
+    return base if world == 1 else base + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (all ranks call it; no-op on one rank)."""
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(flops_per_rank: float, world: int, ms_step: float) -> float:
+    """Weak scaling: every rank did flops_per_rank in at most ms_step (TFLOP/s)."""
+    return flops_per_rank * world / (ms_step * 1e-3) / 1e12
+
+
 def make(args, dev, rank, world):
-    seed_off = 0 if world == 1 else 1000 * rank
     if args.workload == "dense":
-        return DenseWorkload(dev, 2 + seed_off, args.heads)
+        return DenseWorkload(dev, rank_seed(2, rank, world), args.heads)
     if args.workload == "chunked":
-        return ChunkedWorkload(dev, 4 + seed_off, args.heads)
-    return SparseWorkload(dev, 5 + seed_off, args.heads, padded=args.workload == "sparse-padded")
+        return ChunkedWorkload(dev, rank_seed(4, rank, world), args.heads)
+    return SparseWorkload(dev, rank_seed(5, rank, world), args.heads,
+                          padded=args.workload == "sparse-padded")
 
 
 def run_reference(args, rank: int, world: int):
@@ -511,11 +532,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         merge_ms = sum(a.elapsed_time(b) for a, b in w.merge_events) / len(w.merge_events)
         w.merge_events = None
     ms_total = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
-    value = w.flops * world / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(ms_total, world, dev) / args.steps
+    value = whole_job_value(w.flops, world, ms_step)
     status = mla.mla_device_status(reset=True)
     if args.kernel_only:
         if rank == 0:
@@ -537,10 +555,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         w.e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, world, dev)
     h2d = sum(x.numel() * x.element_size() for x in w.hin)
     d2h = sum(x.numel() * x.element_size() for x in w.hout)
 
@@ -565,7 +580,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                      "traffic": recorded_traffic_for(w.profile, w.sources),
                      "kernel": w.kernel,
                      "timed": "one public call per step; CUDA events on its stream"},
-        "e2e": {"value": w.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": whole_job_value(w.flops, world, e2e_ms), "unit": UNIT,
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * w.launches,
         "clocks": clocks,

@@ -123,6 +123,29 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
                     size_t workspace_bytes);
 
 /*
+ * mla_prefill_fwd over strided q, k and v (for example V as a view into a
+ * buffer that interleaves k_nope and v per head, the layout of vLLM's MLA
+ * prefill backend, "Vllm project Vllm FlashAttention MLA Prefill", where v
+ * is a slice with row stride num_heads * (nope + v) and head stride nope + v).
+ *
+ * Element (row r, head h, dim d) of x is at x + r * x_row_stride +
+ * h * x_head_stride + d (bf16 elements; the dim is contiguous).  Each stride
+ * must be positive, a multiple of 8 elements (16 bytes) and below 2^39; the
+ * base pointers stay 16-B aligned.  Rows of different heads may overlap in
+ * memory (the call only reads q, k and v).  All other arguments are those of
+ * mla_prefill_fwd, which is this call with the packed strides
+ * (num_heads * 192, 192) for q and k and (num_heads * 128, 128) for v.
+ * Returns MLA_ERR_INVALID_ARG for a stride the tensor-map encoder refuses.
+ */
+int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride, int64_t k_head_stride,
+                            const void* v, int64_t v_row_stride, int64_t v_head_stride,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                            int total_q, int total_k, void* workspace, size_t workspace_bytes);
+
+/*
  * mla_prefill_fwd for callers that cannot allocate device memory.
  *
  * (The pages have no counterpart to this entry point; it is a convenience of

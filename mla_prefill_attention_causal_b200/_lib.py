@@ -33,13 +33,15 @@ QK_DIM, V_DIM = 192, 128
 LATENT_DIM, LATENT_V_DIM = 576, 512
 
 # name -> (restype, argtypes), mirroring include/mla.h
-_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_P, _I, _F, _S, _L = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_int64
 SIGNATURES = {
     "mla_status_string": (ctypes.c_char_p, [_I]),
     "mla_version": (_I, []),
     "mla_prefill_workspace_size": (_S, [_I, _I]),
     "mla_prefill_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P,
                              _S]),
+    "mla_prefill_fwd_strided": (_I, [_P, _L, _L, _P, _L, _L, _P, _L, _L, _P, _P, _I, _I, _F, _I,
+                                     _P, _P, _P, _I, _I, _I, _I, _P, _S]),
     "mla_prefill_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I,
                                      _I]),
     "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
@@ -93,7 +95,7 @@ def _stream() -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype, ndim: int) -> None:
+def _need(t: torch.Tensor, name: str, dtype, ndim: int, contiguous: bool = True) -> None:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -102,8 +104,12 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int) -> None:
         raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
-    if not t.is_contiguous():
+    if contiguous and not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if not contiguous and (t.stride(-1) != 1 or any(x % 8 for x in t.stride()[:-1])
+                           or t.data_ptr() % 16):
+        raise ValueError(f"{name} needs a contiguous last dim, other strides that are multiples "
+                         f"of 8 elements and a 16-byte aligned start; got strides {t.stride()}")
 
 
 def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -115,14 +121,17 @@ def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     """Dense varlen MLA prefill forward (``mla_prefill_fwd`` in ``mla.h``).
 
     q ``[total_q, H, 192]``, k ``[total_k, H, 192]``, v ``[total_k, H, 128]``
-    (bf16, contiguous, CUDA); cu_seqlens int32 ``[B+1]`` on the same device.
+    (bf16, CUDA; contiguous, or views whose last dim is contiguous and whose
+    other strides are multiples of 8 elements, which go through
+    ``mla_prefill_fwd_strided``); cu_seqlens int32 ``[B+1]`` on the same
+    device.
     ``workspace`` (uint8, >= ``prefill_workspace_size(B, total_q)`` bytes) is
     allocated from PyTorch's stream-ordered allocator when not given.
     Returns ``(out [total_q, H, 128] bf16, lse [H, total_q] fp32 or None)``.
     """
-    _need(q, "q", torch.bfloat16, 3)
-    _need(k, "k", torch.bfloat16, 3)
-    _need(v, "v", torch.bfloat16, 3)
+    _need(q, "q", torch.bfloat16, 3, contiguous=False)
+    _need(k, "k", torch.bfloat16, 3, contiguous=False)
+    _need(v, "v", torch.bfloat16, 3, contiguous=False)
     _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
     _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
     total_q, num_heads, dq = q.shape
@@ -152,12 +161,17 @@ def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     elif workspace.numel() * workspace.element_size() < ws_bytes or not workspace.is_cuda:
         raise ValueError(f"workspace must be a CUDA buffer of >= {ws_bytes} bytes")
-    st = load().mla_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
-                                int(max_seqlen_q), int(max_seqlen_k), float(softmax_scale),
-                                1 if causal else 0, _ptr(out), _ptr(lse), _stream(),
-                                batch, num_heads, total_q, total_k, _ptr(workspace),
-                                workspace.numel() * workspace.element_size())
-    _check("mla_prefill_fwd", st)
+    rest = (_ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
+            float(softmax_scale), 1 if causal else 0, _ptr(out), _ptr(lse), _stream(), batch,
+            num_heads, total_q, total_k, _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    if q.is_contiguous() and k.is_contiguous() and v.is_contiguous():
+        st = load().mla_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), *rest)
+        _check("mla_prefill_fwd", st)
+    else:
+        st = load().mla_prefill_fwd_strided(_ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0),
+                                            k.stride(1), _ptr(v), v.stride(0), v.stride(1), *rest)
+        _check("mla_prefill_fwd_strided", st)
     return out, lse
 
 

@@ -349,8 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qbar = lead(&bars->q_full[i]);
 #pragma unroll
             for (int c = 0; c < kQkChunks; ++c)
-              tma_load_2d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q,
-                               ti.h * kDqk + 64 * c,
+              tma_load_3d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q, 64 * c, ti.h,
                                ti.q_start + ti.m0 + i * kSubRows + static_cast<int>(rank) * kCtaRows,
                                qbar, pol_q);
           } else if (leader) {
@@ -368,9 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kbar = lead(&bars->full_k[slot]);
 #pragma unroll
           for (int u = 0; u < kKUnits; ++u)
-            tma_load_2d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, &tm_k,
-                             ti.h * kDqk + 64 * u, key0 + static_cast<int>(rank) * kHalfKeys, kbar,
-                             pol_kv);
+            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, &tm_k, 64 * u, ti.h,
+                             key0 + static_cast<int>(rank) * kHalfKeys, kbar, pol_kv);
           // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
           if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
@@ -378,9 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t vbar = lead(&bars->full_v[slot]);
 #pragma unroll
           for (int u = 0; u < kVUnits; ++u)
-            tma_load_2d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, &tm_v,
-                             ti.h * kDv + static_cast<int>(rank) * kHalfDv, key0 + 64 * u, vbar,
-                             pol_kv);
+            tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, &tm_v,
+                             static_cast<int>(rank) * kHalfDv, ti.h, key0 + 64 * u, vbar, pol_kv);
         }
       }
       if (!ok && leader) {

@@ -141,6 +141,27 @@ int encode_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// 3-D bf16 tensor map over [rows, heads, dim] with arbitrary row and head
+// strides (elements; the dim is contiguous), a 64-element x 1-head x
+// box_rows box and the 128-byte swizzle.  Rows past `rows` read as zero.
+int encode_heads(CUtensorMap* map, const void* base, uint64_t dim, uint64_t heads, uint64_t rows,
+                 int64_t head_stride, int64_t row_stride, uint32_t box_rows) {
+  const cuuint64_t dims[3] = {dim, heads, rows};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_stride) * 2,
+                                 static_cast<cuuint64_t>(row_stride) * 2};
+  const cuuint32_t box[3] = {64, 1, box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                                 dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
+}
+
+// Strides a TMA map accepts: positive, a multiple of 8 elements (16 bytes)
+// and below 2^39 elements.
+bool good_stride(int64_t st) { return st > 0 && st % 8 == 0 && st < (int64_t{1} << 39); }
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
 // Scratch for mla_prefill_fwd_noalloc: the dense kernels' work list for
@@ -217,6 +238,22 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
                     float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
                     int batch, int num_heads, int total_q, int total_k, void* workspace,
                     size_t workspace_bytes) {
+  using mla::dense::kDqk;
+  using mla::dense::kDv;
+  const int64_t H = num_heads;
+  return mla_prefill_fwd_strided(q, H * kDqk, kDqk, k, H * kDqk, kDqk, v, H * kDv, kDv,
+                                 cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                                 softmax_scale, causal, out, lse, stream, batch, num_heads,
+                                 total_q, total_k, workspace, workspace_bytes);
+}
+
+int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride, int64_t k_head_stride,
+                            const void* v, int64_t v_row_stride, int64_t v_head_stride,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                            int total_q, int total_k, void* workspace, size_t workspace_bytes) {
   using namespace mla::dense;
   if (q == nullptr || k == nullptr || v == nullptr || cu_seqlens_q == nullptr ||
       cu_seqlens_k == nullptr || out == nullptr || workspace == nullptr)
@@ -229,6 +266,9 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
       max_seqlen_q < 0 || max_seqlen_k < 0 || (causal != 0 && causal != 1))
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  if (!good_stride(q_row_stride) || !good_stride(q_head_stride) || !good_stride(k_row_stride) ||
+      !good_stride(k_head_stride) || !good_stride(v_row_stride) || !good_stride(v_head_stride))
+    return MLA_ERR_INVALID_ARG;
   const size_t need = mla_prefill_workspace_size(batch, total_q);
   if (workspace_bytes < need) return MLA_ERR_INVALID_ARG;
   int dev = 0;
@@ -238,11 +278,12 @@ int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* 
 
   CUtensorMap tq, tk, tv;
   const uint64_t kv_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
-  if ((st = encode_rows(&tq, q, static_cast<uint64_t>(num_heads) * kDqk, total_q, kCtaRows)) !=
+  const uint64_t H = static_cast<uint64_t>(num_heads);
+  if ((st = encode_heads(&tq, q, kDqk, H, static_cast<uint64_t>(total_q), q_head_stride,
+                         q_row_stride, kCtaRows)) != MLA_OK ||
+      (st = encode_heads(&tk, k, kDqk, H, kv_rows, k_head_stride, k_row_stride, kHalfKeys)) !=
           MLA_OK ||
-      (st = encode_rows(&tk, k, static_cast<uint64_t>(num_heads) * kDqk, kv_rows, kHalfKeys)) !=
-          MLA_OK ||
-      (st = encode_rows(&tv, v, static_cast<uint64_t>(num_heads) * kDv, kv_rows, 64)) != MLA_OK)
+      (st = encode_heads(&tv, v, kDv, H, kv_rows, v_head_stride, v_row_stride, 64)) != MLA_OK)
     return st;
 
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

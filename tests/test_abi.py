@@ -98,3 +98,17 @@ def test_python_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libmla.so")
     with pytest.raises(RuntimeError, match="not built"):
         _lib.load()
+
+
+def _call_strided(qs=(64, 32), ks=(64, 32), vs=(64, 32)):
+    P = ctypes.c_void_p
+    return mla.load().mla_prefill_fwd_strided(
+        P(16), qs[0], qs[1], P(16), ks[0], ks[1], P(16), vs[0], vs[1], P(16), P(16), 4, 4, 0.1, 1,
+        P(16), None, None, 1, 1, 4, 4, P(64), 4096)
+
+
+@pytest.mark.parametrize("bad", [dict(qs=(0, 32)), dict(ks=(64, -8)), dict(vs=(60, 32)),
+                                 dict(qs=(64, 12)), dict(vs=(1 << 40, 32))])
+def test_strided_rejects_bad_strides(bad):
+    # checked on the host before the device is touched
+    assert _call_strided(**bad) == _lib.MLA_ERR_INVALID_ARG

@@ -92,6 +92,37 @@ def test_batch_invariant():
     assert torch.equal(l1, l_all[:, s0:s1])
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_strided_views_match_packed_inputs(causal):
+    """q, k, v as views into wider buffers (v interleaved with k_nope per head,
+    as in vLLM's MLA prefill backend) give the packed call's result exactly."""
+    import mla_prefill_attention_causal_b200 as mla
+    case = syn.dense_case([300, 129, 1], [300, 129, 1] if causal else [513, 64, 200], 4, seed=77,
+                          causal=causal)
+    q, k, v = dev_bf16(case["q"]), dev_bf16(case["k"]), dev_bf16(case["v"])
+    cq, ck = dev_i32(case["cu_q"]), dev_i32(case["cu_k"])
+    T, H = q.shape[0], q.shape[1]
+    Tk = k.shape[0]
+    qbuf = torch.zeros((T, H, 256), dtype=torch.bfloat16, device="cuda")
+    qbuf[..., :192] = q                       # head stride 256
+    kbuf = torch.zeros((Tk, H + 1, 192), dtype=torch.bfloat16, device="cuda")
+    kbuf[:, :H] = k                           # row stride (H + 1) * 192
+    kv = torch.zeros((Tk, H, 256), dtype=torch.bfloat16, device="cuda")
+    kv[..., 128:] = v                         # v = kv[..., 128:]: head stride 256, offset 256 B
+    qs, ks, vs = qbuf[..., :192], kbuf[:, :H], kv[..., 128:]
+    assert not (qs.is_contiguous() or ks.is_contiguous() or vs.is_contiguous())
+    a = mla.mla_prefill_fwd(q, k, v, cq, ck, case["max_q"], case["max_k"], case["scale"],
+                            causal=causal)
+    b = mla.mla_prefill_fwd(qs, ks, vs, cq, ck, case["max_q"], case["max_k"], case["scale"],
+                            causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    ref_o, ref_l = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"],
+                                        case["cu_k"], case["scale"], causal)
+    assert_out_close(to_f64(b[0]), ref_o)
+    assert_lse_close(b[1].cpu().numpy().astype(np.float64), ref_l)
+
+
 def test_many_heads_small():
     lens = [383, 129]
     check_dense(syn.dense_case(lens, lens, 128, seed=18))

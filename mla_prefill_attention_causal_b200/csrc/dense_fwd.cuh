@@ -98,8 +98,7 @@ struct TileInfo {
 struct alignas(8) Bars {
   uint64_t q_full[2];    // leader: Q bytes of both CTAs
   uint64_t q_empty[2];   // both: last S MMA of the tile done
-  uint64_t full_k[kSlots];   // leader: K-half bytes of both CTAs
-  uint64_t full_v[kSlots];   // leader: V-half bytes of both CTAs
+  uint64_t full_kv[kSlots];  // leader: K- and V-half bytes of block b, both CTAs
   uint64_t empty_k[kSlots];  // both: the S MMAs reading the K slot done
   uint64_t empty_v[kSlots];  // both: the PV MMAs reading the V slot done
   uint64_t s_full[2];    // both
@@ -296,8 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->o_empty[i]), 8);
     }
     for (int i = 0; i < kSlots; ++i) {
-      mbar_init(smem_u32(&bars->full_k[i]), 1);
-      mbar_init(smem_u32(&bars->full_v[i]), 1);
+      mbar_init(smem_u32(&bars->full_kv[i]), 1);
       mbar_init(smem_u32(&bars->empty_k[i]), 1);
       mbar_init(smem_u32(&bars->empty_v[i]), 1);
     }
@@ -363,8 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // K: this CTA's 64 keys, three 64-dim chunks of the 192
           if (!(ok = wait(smem_u32(&bars->empty_k[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full_k[slot]), 2 * kKSlotBytes);
-          const uint32_t kbar = lead(&bars->full_k[slot]);
+          // one barrier per block for K and V: the MMA warp waits once per block
+          if (leader)
+            mbar_arrive_expect_tx(smem_u32(&bars->full_kv[slot]), 2 * (kKSlotBytes + kVSlotBytes));
+          const uint32_t kbar = lead(&bars->full_kv[slot]);
 #pragma unroll
           for (int u = 0; u < kKUnits; ++u)
             tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, &tm_k, 64 * u, ti.h,
@@ -372,8 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
           if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full_v[slot]), 2 * kVSlotBytes);
-          const uint32_t vbar = lead(&bars->full_v[slot]);
+          const uint32_t vbar = kbar;
 #pragma unroll
           for (int u = 0; u < kVUnits; ++u)
             tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, &tm_v,
@@ -385,8 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int no_abort = 0;
         for (int b = max(0, blk - kSlots); b <= blk; ++b) {
           const uint32_t par = static_cast<uint32_t>(b / kSlots) & 1u;
-          mbar_wait(smem_u32(&bars->full_k[b % kSlots]), par, &no_abort, 0, tlim / 8);
-          mbar_wait(smem_u32(&bars->full_v[b % kSlots]), par, &no_abort, 0, tlim / 8);
+          mbar_wait(smem_u32(&bars->full_kv[b % kSlots]), par, &no_abort, 0, tlim / 8);
         }
       }
     }
@@ -399,11 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return r;
       };
-      auto wait_k = [&](int b) -> bool {
-        return wait_bar(smem_u32(&bars->full_k[b % kSlots]), static_cast<uint32_t>(b / kSlots) & 1u);
-      };
-      auto wait_v = [&](int b) -> bool {
-        return wait_bar(smem_u32(&bars->full_v[b % kSlots]), static_cast<uint32_t>(b / kSlots) & 1u);
+      // K and V of block b (one barrier); V(b) is covered by the wait that
+      // preceded S(b).
+      auto wait_kv = [&](int b) -> bool {
+        return wait_bar(smem_u32(&bars->full_kv[b % kSlots]), static_cast<uint32_t>(b / kSlots) & 1u);
       };
       auto commit_both = [&](uint64_t* bar) { tc_commit_pair_elect(smem_u32(bar), 0x3); };
       // Descriptors: built once per burst, then advanced by adding to the
@@ -439,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i)
           if (!wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k) & 1u)) return false;
         if (max(n[0], n[1]) > 0) {
-          if (!wait_k(b)) return false;
+          if (!wait_kv(b)) return false;
           for (int i = 0; i < 2; ++i) {
             if (n[i] > 0) issue_s(i, b);
             if (n[i] <= 1) commit_both(&bars->q_empty[i]);
@@ -464,14 +461,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = 0; n < nblk && ok; ++n) {
           const int b = blk + n;  // this KV block; the next one is b + 1
           const bool last = n + 1 == nblk;
-          if (!(ok = wait_v(b))) break;
           bool next_s[2] = {n + 1 < nb[0], n + 1 < nb[1]};
           if (last) {
             next_s[0] = nbn[0] > 0;
             next_s[1] = nbn[1] > 0;
           }
           const bool more = next_s[0] || next_s[1];
-          if (more && !(ok = wait_k(b + 1))) break;
+          if (more && !(ok = wait_kv(b + 1))) break;
           for (int i = 0; i < 2 && ok; ++i) {
             if (n < nb[i]) {
               if (n == 0 && !(ok = wait_bar(smem_u32(&bars->o_empty[i]),

@@ -590,8 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            // 10 of every 16 pairs on the MUFU unit, 6 on the FMA pipe
-            if ((j & 7) < 5)
+            // 14 of every 16 pairs on the MUFU unit, 2 on the FMA pipe
+            if ((j & 7) < 7)
               pk[j] = softmax_pair_mufu(x[32 * c + 2 * j], x[32 * c + 2 * j + 1], c2, negm2,
                                         acc[j & 3]);
             else

@@ -69,6 +69,7 @@ struct alignas(8) Bars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int last_valid;           // position of the token's last valid slot (-1: none)
 };
 
 constexpr int kSmemBytes = 1024 + kQsBytes + kSlots * kSlotBytes + static_cast<int>(sizeof(Bars));
@@ -98,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int t = static_cast<int>(blockIdx.x >> 1);
   const int half = static_cast<int>(blockIdx.x & 1);
-  const int nchunks = (p.topk + kChunk - 1) / kChunk;
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&bars->o_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
+    bars->last_valid = -1;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -136,6 +137,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto warp_wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, tlim));
   };
+
+  // Prologue.  Q dims 256-575 go to shared memory by TMA and the softmax
+  // warps write Q dims 0-255 into TMEM; meanwhile the other warps find the
+  // last valid slot of the token's index list.  Chunks after it hold only
+  // padding and are not processed (left-aligned lists with -1 fill, the
+  // common layout, then skip all their padding; padding elsewhere is masked).
+  if (warp == kMmaWarp && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
+    for (int c = 0; c < kQsChunks; ++c)
+      tma_load_2d_hint(sQ + c * kQChunkBytes, &tm_q, kQtDims + 64 * c, t * p.num_heads,
+                       smem_u32(&bars->q_full), l2_policy_evict_first());
+  }
+  if (warp < 4) {
+    // Q dims 0-255 of this head as bf16 pairs in TMEM columns [kColQ, +128)
+    const int h = threadIdx.x;
+    const bool row_ok = h < p.num_heads;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint4* qrow = reinterpret_cast<const uint4*>(
+        p.q + (static_cast<size_t>(t) * p.num_heads + (row_ok ? h : 0)) * kDl);
+#pragma unroll
+    for (int c = 0; c < kQtDims / 32; ++c) {  // 32 dims = 16 columns per store
+      uint32_t v[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = row_ok ? __ldg(qrow + 4 * c + i) : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * i] = w.x;
+        v[4 * i + 1] = w.y;
+        v[4 * i + 2] = w.z;
+        v[4 * i + 3] = w.w;
+      }
+      tmem_st_x16(tmem + lane_off + kColQ + 16 * c, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->qt_ready));
+  } else {
+    // Each warp walks its positions from the end of the list backwards and
+    // stops at its first valid slot (the largest of its positions), so an
+    // unpadded list costs one load per thread.
+    const int* idx_row = p.indices + static_cast<size_t>(t) * p.topk;
+    constexpr int kScanThreads = kThreads - 128;
+    const int r = static_cast<int>(threadIdx.x) - 128;
+    int last = -1;
+    for (int base = p.topk - kScanThreads; base > -kScanThreads; base -= kScanThreads) {
+      const int i = base + r;
+      int hit = -1;
+      if (i >= 0) {
+        const int v = __ldg(idx_row + i);
+        if (v >= 0 && v < p.num_rows) hit = i;
+      }
+      hit = __reduce_max_sync(0xffffffffu, hit);
+      if (hit >= 0) {
+        last = hit;
+        break;
+      }
+    }
+    if (lane == 0 && last >= 0) atomicMax(&bars->last_valid, last);
+  }
+  __syncthreads();
+  const int nchunks = (bars->last_valid + kChunk) / kChunk;  // chunks up to the last valid slot
 
   if (warp >= 4 && warp < kMmaWarp) {
     // ------------------------------------------------------------ loaders
@@ -211,14 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_elect(smem_u32(&bars->pv_done));
       tc_commit_elect(smem_u32(&bars->empty[c % kSlots]));
     };
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kQsBytes);
-      for (int c = 0; c < kQsChunks; ++c)
-        tma_load_2d_hint(sQ + c * kQChunkBytes, &tm_q, kQtDims + 64 * c, t * p.num_heads,
-                         smem_u32(&bars->q_full), l2_policy_evict_first());
-    }
-    __syncwarp();
     ok = wait_bar(smem_u32(&bars->q_full), 0) && wait_bar(smem_u32(&bars->qt_ready), 0);
     // Issue S(c) and PV(c) in whichever order their inputs arrive: PV(c)
     // frees chunk c's slot for the next gather, so it must not queue behind
@@ -277,28 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = threadIdx.x;  // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const bool row_ok = h < p.num_heads;
-    // Q dims 0-255 of this head as bf16 pairs in TMEM columns [kColQ, +128)
-    {
-      const uint4* qrow = reinterpret_cast<const uint4*>(
-          p.q + (static_cast<size_t>(t) * p.num_heads + (row_ok ? h : 0)) * kDl);
-#pragma unroll
-      for (int c = 0; c < kQtDims / 32; ++c) {  // 32 dims = 16 columns per store
-        uint32_t v[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 w = row_ok ? __ldg(qrow + 4 * c + i) : make_uint4(0u, 0u, 0u, 0u);
-          v[4 * i] = w.x;
-          v[4 * i + 1] = w.y;
-          v[4 * i + 2] = w.z;
-          v[4 * i + 3] = w.w;
-        }
-        tmem_st_x16(tmem + lane_off + kColQ + 16 * c, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->qt_ready));
-    }
     const float sl2 = p.scale_log2;
     const uint64_t c2 = pack_f32x2(sl2, sl2);
     const Exp2PolyConsts pk2 = exp2_poly_consts();
@@ -405,9 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v4 = 0; v4 < 4; ++v4) {
             uint32_t pk[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
-                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv);
+            for (int j = 0; j < 4; ++j)  // no valid slot: O = 0 (TMEM O may be unwritten)
+              pk[j] = seen ? pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
+                                         __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv)
+                           : 0u;
             orow[4 * q + v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }

@@ -33,8 +33,10 @@
 // dims), a K ring of 3 slots (this CTA's 64 keys x 192 dims = 3 units of
 // 64 rows x 64 dims, 24 KB) and a V ring of 3 slots (128 keys x this CTA's
 // 64 dims = 2 units, 16 KB), all with the 128-byte swizzle used by TMA and
-// the MMA descriptors.  One barrier per slot and direction: K(b) is freed
-// after both S MMAs of block b, V(b) after both PV MMAs.
+// the MMA descriptors.  K(b) and V(b) land on one barrier (the MMA warp
+// waits once per block); K(b) is freed after both S MMAs of block b, V(b)
+// after both PV MMAs.  Q, K and V are read through 3-D (dim, head, row)
+// tensor maps, so strided views need no copies.
 // TMEM per CTA (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1
 // [384,512); P_i (bf16, 64 columns) overwrites the first half of S_i.
 //

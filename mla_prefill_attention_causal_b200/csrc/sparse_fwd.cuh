@@ -26,8 +26,9 @@
 //               memory
 // TMEM (512 columns): S buffers [0,64) and [64,128) (P overwrites their
 // first 32 columns), Q dims 0-255 as bf16 pairs [128,256), O [256,512).
-// MMA order: S(0), S(1), PV(0), S(2), PV(1), ... (S of the next chunk runs
-// while the current chunk's softmax does).
+// MMAs are issued as their inputs arrive; S of the next chunk runs while
+// the current chunk's softmax does.  Chunks after the token's last valid
+// slot are not processed.
 #pragma once
 #include <cuda_bf16.h>
 

@@ -112,3 +112,23 @@ def _call_strided(qs=(64, 32), ks=(64, 32), vs=(64, 32)):
 def test_strided_rejects_bad_strides(bad):
     # checked on the host before the device is touched
     assert _call_strided(**bad) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_python_binding_checks_arguments_before_any_launch():
+    import torch
+    q = torch.zeros((4, 2, 192), dtype=torch.bfloat16)
+    k = torch.zeros((4, 2, 192), dtype=torch.bfloat16)
+    v = torch.zeros((4, 2, 128), dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA device"):
+        mla.mla_prefill_fwd(q, k, v, cu, cu, 4, 4)
+    with pytest.raises(TypeError, match="bfloat16"):
+        mla.mla_prefill_fwd(q.float(), k, v, cu, cu, 4, 4)
+    with pytest.raises(ValueError, match="3 dims"):
+        mla.mla_prefill_fwd(q[0], k, v, cu, cu, 4, 4)
+    kv = torch.zeros((4, 576), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        mla.mla_sparse_prefill_fwd(torch.zeros((4, 8, 576), dtype=torch.bfloat16), kv,
+                                   torch.zeros((4, 16), dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA device"):
+        mla.mla_attn_merge(v, torch.zeros((2, 4)), v, torch.zeros((2, 4)))

@@ -70,8 +70,8 @@ int mla_version(void);
 
 /*
  * Bytes of device workspace mla_prefill_fwd needs for a call with these
- * sizes: a small header plus one 8-byte entry per (sequence, 256-row query
- * block), at most ceil(total_q / 256) + batch of them.  Returns 0 for
+ * sizes: a small header plus one 8-byte entry per (sequence, 512-row query
+ * block), at most ceil(total_q / 512) + batch of them.  Returns 0 for
  * invalid sizes.
  */
 size_t mla_prefill_workspace_size(int batch, int total_q);

@@ -228,8 +228,9 @@ int mla_version(void) { return 100; }
 
 size_t mla_prefill_workspace_size(int batch, int total_q) {
   if (batch < 1 || total_q < 0) return 0;
-  const size_t entries = static_cast<size_t>((total_q + mla::dense::kTileRows - 1) /
-                                             mla::dense::kTileRows) + static_cast<size_t>(batch);
+  const size_t entries =
+      (static_cast<size_t>(total_q) + mla::dense::kTileRows - 1) / mla::dense::kTileRows +
+      static_cast<size_t>(batch);
   return mla::dense::kWsHeaderBytes + entries * sizeof(int2);
 }
 
@@ -271,6 +272,9 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
     return MLA_ERR_INVALID_ARG;
   const size_t need = mla_prefill_workspace_size(batch, total_q);
   if (workspace_bytes < need) return MLA_ERR_INVALID_ARG;
+  // the kernels count tiles (work-list entries x heads) in int
+  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * num_heads > INT32_MAX)
+    return MLA_ERR_INVALID_ARG;
   int dev = 0;
   int st = prepare_device(&dev);
   if (st != MLA_OK) return st;

@@ -67,6 +67,15 @@ def test_dense_rejects_bad_arguments(over):
     assert _call_dense(**over) == _lib.MLA_ERR_INVALID_ARG
 
 
+def test_dense_rejects_tile_counts_beyond_int():
+    # 2^31 - 1 query rows x 65535 heads: the workspace is big enough, but the
+    # number of (512-row block, head) tiles does not fit the kernels' int
+    tq, H = 2**31 - 1, 65535
+    need = mla.prefill_workspace_size(1, tq)
+    assert need > 0
+    assert _call_dense(tq=tq, H=H, wsb=need) == _lib.MLA_ERR_INVALID_ARG
+
+
 def test_merge_rejects_bad_arguments():
     f = mla.load().mla_attn_merge
     P = ctypes.c_void_p

@@ -112,6 +112,12 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int, contiguous: bool = True)
                          f"of 8 elements and a 16-byte aligned start; got strides {t.stride()}")
 
 
+def _same_device(ref: torch.Tensor, **tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, the inputs on {ref.device}")
+
+
 def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
                     max_seqlen_q: int, max_seqlen_k: int,
@@ -161,6 +167,16 @@ def mla_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     elif workspace.numel() * workspace.element_size() < ws_bytes or not workspace.is_cuda:
         raise ValueError(f"workspace must be a CUDA buffer of >= {ws_bytes} bytes")
+    _same_device(q, k=k, v=v, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, out=out,
+                 lse=lse, workspace=workspace)
+    with torch.cuda.device(q.device):
+        return _prefill_call(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                             softmax_scale, causal, out, lse, batch, num_heads, total_q, total_k,
+                             workspace)
+
+
+def _prefill_call(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale,
+                  causal, out, lse, batch, num_heads, total_q, total_k, workspace):
     rest = (_ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
             float(softmax_scale), 1 if causal else 0, _ptr(out), _ptr(lse), _stream(), batch,
             num_heads, total_q, total_k, _ptr(workspace),
@@ -199,10 +215,18 @@ def mla_attn_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor,
         out = torch.empty_like(o_a)
     else:
         _need(out, "out", torch.bfloat16, 3)
+        if out.shape != o_a.shape:
+            raise ValueError("out must have the partial results' shape")
     if lse_out is None and return_lse:
         lse_out = torch.empty_like(lse_a)
-    st = load().mla_attn_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
-                               _ptr(lse_out), T, H, D, _stream())
+    elif lse_out is not None:
+        _need(lse_out, "lse_out", torch.float32, 2)
+        if lse_out.shape != (H, T):
+            raise ValueError("lse_out must be [num_heads, num_tokens]")
+    _same_device(o_a, o_b=o_b, lse_a=lse_a, lse_b=lse_b, out=out, lse_out=lse_out)
+    with torch.cuda.device(o_a.device):
+        st = load().mla_attn_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
+                                   _ptr(lse_out), T, H, D, _stream())
     _check("mla_attn_merge", st)
     return out, lse_out
 
@@ -229,13 +253,27 @@ def mla_sparse_prefill_fwd(q: torch.Tensor, kv_latent: torch.Tensor, indices: to
         softmax_scale = 1.0 / math.sqrt(LATENT_DIM)
     if out is None:
         out = torch.empty((T, H, LATENT_V_DIM), dtype=torch.bfloat16, device=q.device)
+    else:
+        _need(out, "out", torch.bfloat16, 3)
+        if out.shape != (T, H, LATENT_V_DIM):
+            raise ValueError(f"out must be [T, H, {LATENT_V_DIM}]")
     if lse is None and return_lse:
         lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
-    st = load().mla_sparse_prefill_fwd(_ptr(q), _ptr(kv_latent), _ptr(indices), topk,
-                                       float(softmax_scale), _ptr(out), _ptr(lse), _stream(),
-                                       T, H, N)
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+        if lse.shape != (H, T):
+            raise ValueError("lse must be [num_heads, num_tokens]")
+    _same_device(q, kv_latent=kv_latent, indices=indices, out=out, lse=lse)
+    with torch.cuda.device(q.device):
+        st = _sparse_call(q, kv_latent, indices, topk, softmax_scale, out, lse, T, H, N)
     _check("mla_sparse_prefill_fwd", st)
     return out, lse
+
+
+def _sparse_call(q, kv_latent, indices, topk, softmax_scale, out, lse, T, H, N):
+    return load().mla_sparse_prefill_fwd(_ptr(q), _ptr(kv_latent), _ptr(indices), topk,
+                                       float(softmax_scale), _ptr(out), _ptr(lse), _stream(),
+                                       T, H, N)
 
 
 def mla_device_status(reset: bool = True) -> int:

@@ -62,6 +62,19 @@ def test_warmup_probe_shapes(max_q, max_k, causal):
     check_dense(case)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_large_scores_rescale_the_running_max(causal):
+    """q x 32 (exact: a power of two): scores with a standard deviation of 32
+    make rows' running maxima jump by more than the lazy threshold in later
+    KV blocks, so the O rescale path runs (N(0,1) data almost never takes it)."""
+    lens_q = [700, 300, 129]
+    lens_k = lens_q if causal else [900, 300, 400]
+    case = syn.dense_case(lens_q, lens_k, 4, seed=71, causal=causal)
+    widened = (case["q"].astype(np.uint32) << np.uint32(16)).view(np.float32)
+    case = dict(case, q=syn.f32_to_bf16_bits(widened * np.float32(32.0)))
+    check_dense(case)
+
+
 def test_lse_optional_and_out_identical():
     case = syn.dense_case([300, 77], [300, 77], 2, seed=15)
     o1, l1 = run_dense(case, want_lse=True)

@@ -357,6 +357,19 @@ def test_flop_counts():
     assert oracle.sparse_flops(idx, 10, 4) == 2 * (576 + 512) * 4 * 3
 
 
+def test_flop_counts_match_the_counted_mask():
+    """The FLOP numerator of every TFLOP/s figure: visible (query, key) pairs
+    counted on an explicit bottom-right mask matrix (numpy's tril with the
+    diagonal offset Lk - Lq) for square and ragged shapes."""
+    g = np.random.Generator(np.random.PCG64(11))
+    shapes = [(1, 1), (1, 300), (300, 1), (128, 128), (129, 127), (512, 4096), (4096, 512)]
+    shapes += [tuple(int(x) for x in g.integers(0, 700, size=2)) for _ in range(20)]
+    for lq, lk in shapes:
+        mask = np.tril(np.ones((lq, lk), dtype=np.int64), k=lk - lq)
+        assert oracle.dense_flops([lq], [lk], 3, True) == 2 * 320 * 3 * int(mask.sum()), (lq, lk)
+        assert oracle.dense_flops([lq], [lk], 3, False) == 2 * 320 * 3 * lq * lk
+
+
 # ---------------------------------------------------------------------------
 # Mutation tests: plant a mistake in the oracle; some pin must fail.
 # ---------------------------------------------------------------------------

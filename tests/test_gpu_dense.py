@@ -141,6 +141,14 @@ def test_many_heads_small():
     check_dense(syn.dense_case(lens, lens, 128, seed=18))
 
 
+def test_thousands_of_heads_on_tiny_sequences():
+    """4096 heads (tensor-parallel layouts keep fewer, but the head is the
+    slowest index of the work list and of the tensor maps' middle dimension)
+    over sequences of 3, 1 and 130 tokens: 12 288 tiles of mostly empty rows."""
+    lens = [3, 1, 130]
+    check_dense(syn.dense_case(lens, lens, 4096, seed=19))
+
+
 def test_varlen16k_config_sampled():
     """8 sequences, lengths U[512,4096], 128 heads: sampled rows, all heads."""
     case = syn.varlen16k_config()

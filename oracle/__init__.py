@@ -12,11 +12,18 @@ Functions (all pinned by tests in ``tests/test_oracle_pins.py``):
 * ``attn_merge``      -- log-sum-exp merge of two partial results.
 * ``sparse_prefill``  -- absorbed top-k sparse attention over a shared
   latent cache.
+* ``dense_prefill_sinks`` -- ``dense_prefill`` with one attention-sink logit
+  per head.
+* ``e4m3_quantize`` / ``e4m3_decode`` -- the FP8 (e4m3) output encoding
+  with a static scale.
 """
 from .attention import (  # noqa: F401
     bf16_bits_to_f64,
     visible_key_count,
     dense_prefill,
+    dense_prefill_sinks,
+    e4m3_decode,
+    e4m3_quantize,
     attn_merge,
     sparse_prefill,
     dense_flops,

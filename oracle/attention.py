@@ -34,6 +34,17 @@ the repository's design notes):
 * sparse: any index ``< 0`` or ``>= num_rows`` is padding; each slot counts
   once; V is the first 512 of the 576 latent dims;
 * merge: the log-sum-exp identity; a ``-inf`` side has weight 0.
+* attention sinks (FA4 interface feature list: "learnable sink tokens";
+  SparseFlashMla "sinks"; Mojo ``attn_sink_ptr``; the arithmetic is not
+  given): one logit ``s_h`` per head, in the units of the scaled scores,
+  that joins each row's softmax with a zero value -- ``O = sum_j e^x_j v_j /
+  (e^s_h + sum_j e^x_j)`` -- and counts in the LSE; a row with no visible
+  key gets ``O = 0`` and ``LSE = s_h``;
+* FP8 static output scale (vLLM ``supports_quant_output``:
+  ``kFp8StaticTensorSym``; ``output_scale``): the output is
+  ``e4m3(O / output_scale)``, rounded to nearest even and saturated to the
+  largest finite e4m3 value, 448 (the static symmetric scheme clamps to
+  the format's range).
 
 Everything is computed in float64 from the exact bf16 inputs.  There is no
 tiling and no online softmax: each row takes its maximum, then its sum.
@@ -140,6 +151,71 @@ def dense_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale: float,
                     lse[h, dst] = np.where(has, row_max + np.log(np.where(has, z, 1.0)),
                                            -np.inf)
     return out, lse
+
+
+def dense_prefill_sinks(q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale: float,
+                        causal: bool, sinks, rows=None):
+    """``dense_prefill`` with one attention-sink logit per head.
+
+    Each row's softmax runs over its visible keys' scaled scores and the
+    head's sink logit ``sinks[h]``; the sink has no value.  Returns ``(out,
+    lse)`` like ``dense_prefill``: ``lse = log(e^s_h + sum_j e^x_j)``, and a
+    row without visible keys gets ``out = 0``, ``lse = s_h``.
+    """
+    cu_q = np.asarray(cu_seqlens_q, dtype=np.int64)
+    cu_k = np.asarray(cu_seqlens_k, dtype=np.int64)
+    sk = np.asarray(sinks, dtype=np.float64)
+    total_q, num_heads, _ = q.shape
+    dv = v.shape[2]
+    sel_rows = np.arange(total_q) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    out = np.zeros((sel_rows.size, num_heads, dv))
+    lse = np.zeros((num_heads, sel_rows.size))
+    seq_of = np.searchsorted(cu_q, sel_rows, side="right") - 1
+    for n, (r, b) in enumerate(zip(sel_rows, seq_of)):
+        q0, k0, k1 = int(cu_q[b]), int(cu_k[b]), int(cu_k[b + 1])
+        lq, lk = int(cu_q[b + 1]) - q0, k1 - k0
+        cnt = visible_key_count(int(r) - q0, lq, lk, causal)
+        for h in range(num_heads):
+            x = float(softmax_scale) * (_as_f64(k[k0:k0 + cnt, h, :]) @ _as_f64(q[r, h, :]))
+            m = max(float(x.max()) if cnt else -np.inf, sk[h])
+            e = np.exp(x - m)
+            z = float(e.sum()) + np.exp(sk[h] - m)
+            out[n, h, :] = (e @ _as_f64(v[k0:k0 + cnt, h, :])) / z if cnt else 0.0
+            lse[h, n] = m + np.log(z)
+    return out, lse
+
+
+def e4m3_decode(codes):
+    """Values of e4m3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits; exponent 0 is subnormal, m * 2^-9; 0x7F and 0xFF are NaN, there is
+    no infinity)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return sign * val
+
+
+def e4m3_quantize(x, scale: float):
+    """e4m3 codes of ``x / scale``: round to nearest (ties to an even
+    mantissa) on the format's grid -- spacing 2^(e - 3) in binade
+    [2^e, 2^(e+1)), e >= -6, and 2^-9 below 2^-6 -- and saturate at +-448."""
+    y = np.asarray(x, dtype=np.float64) / float(scale)
+    a = np.minimum(np.abs(y), 448.0)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    quantum = np.exp2(e - 3.0)
+    steps = np.round(a / quantum)          # numpy rounds halves to even
+    v = np.minimum(steps * quantum, 448.0)
+    # code of v: normal values as (exponent, mantissa), subnormals below 2^-6
+    ev = np.floor(np.log2(np.where(v > 0, v, 1.0)))
+    normal = v >= 2.0 ** -6
+    mant = np.where(normal, np.round(v / np.exp2(ev) * 8.0) - 8.0, np.round(v / 2.0 ** -9))
+    expo = np.where(normal, ev + 7.0, 0.0)
+    code = (expo.astype(np.int64) << 3) | mant.astype(np.int64)
+    return np.where(y < 0, code | 0x80, code).astype(np.uint8)
 
 
 def attn_merge(o_a, lse_a, o_b, lse_b):

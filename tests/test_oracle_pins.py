@@ -371,6 +371,96 @@ def test_flop_counts_match_the_counted_mask():
 
 
 # ---------------------------------------------------------------------------
+# Attention sinks and the e4m3 output encoding
+# ---------------------------------------------------------------------------
+
+def _sink_case(seed=61, lens=(5, 1, 9), heads=3, causal=True):
+    g = np.random.Generator(np.random.PCG64(seed))
+    lens = list(lens)
+    tq = sum(lens)
+    q = g.standard_normal((tq, heads, 192))
+    k = g.standard_normal((tq, heads, 192))
+    v = g.standard_normal((tq, heads, 128))
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    sinks = g.standard_normal(heads) * 2.0
+    return q, k, v, cu, 1.0 / np.sqrt(192), causal, sinks
+
+
+def pin_sinks_minus_inf_is_no_sink():
+    q, k, v, cu, sc, causal, _ = _sink_case()
+    o, l = oracle.dense_prefill_sinks(q, k, v, cu, cu, sc, causal, np.full(3, -np.inf))
+    o0, l0 = oracle.dense_prefill(q, k, v, cu, cu, sc, causal)
+    assert np.allclose(o, o0, atol=1e-12) and np.allclose(l, l0, atol=1e-12)
+
+
+def pin_sinks_single_key_closed_form():
+    # causal row 0 of each sequence sees one key: O = v0 e^x0 / (e^x0 + e^s)
+    q, k, v, cu, sc, causal, sinks = _sink_case()
+    o, l = oracle.dense_prefill_sinks(q, k, v, cu, cu, sc, True, sinks)
+    for b in range(len(cu) - 1):
+        r = int(cu[b])
+        for h in range(3):
+            x = sc * float(q[r, h] @ k[r, h])
+            w = np.exp(x) / (np.exp(x) + np.exp(sinks[h]))
+            assert np.allclose(o[r, h], w * v[r, h], atol=1e-12)
+            assert abs(l[h, r] - np.log(np.exp(x) + np.exp(sinks[h]))) < 1e-12
+
+
+def pin_sinks_row_without_keys():
+    q, k, v, _, sc, _, sinks = _sink_case()
+    cu_q, cu_k = np.array([0, 4]), np.array([0, 0])  # no keys at all
+    o, l = oracle.dense_prefill_sinks(q[:4], k[:0], v[:0], cu_q, cu_k, sc, True, sinks)
+    assert np.all(o == 0) and np.allclose(l, sinks[:, None].repeat(4, axis=1))
+
+
+def pin_sinks_are_a_zero_valued_extra_key():
+    # the sink merges like a partial result with O = 0 and LSE = s_h
+    q, k, v, cu, sc, causal, sinks = _sink_case(causal=False)
+    o, l = oracle.dense_prefill_sinks(q, k, v, cu, cu, sc, False, sinks)
+    o0, l0 = oracle.dense_prefill(q, k, v, cu, cu, sc, False)
+    om, lm = oracle.attn_merge(o0, l0, np.zeros_like(o0), np.repeat(sinks[:, None], o0.shape[0], 1))
+    assert np.allclose(o, om, atol=1e-12) and np.allclose(l, lm, atol=1e-12)
+
+
+SINK_PINS = [pin_sinks_minus_inf_is_no_sink, pin_sinks_single_key_closed_form,
+             pin_sinks_row_without_keys, pin_sinks_are_a_zero_valued_extra_key]
+
+
+@pytest.mark.parametrize("pin", SINK_PINS, ids=lambda f: f.__name__)
+def test_sink_pin(pin):
+    pin()
+
+
+def test_e4m3_every_finite_code_round_trips():
+    codes = np.arange(256)
+    vals = oracle.e4m3_decode(codes)
+    finite = ~np.isnan(vals)
+    assert finite.sum() == 254  # 0x7F and 0xFF are NaN
+    assert np.array_equal(oracle.e4m3_decode(oracle.e4m3_quantize(vals[finite], 1.0)), vals[finite])
+    assert vals[finite].max() == 448.0 and oracle.e4m3_decode([0x01])[0] == 2.0 ** -9
+
+
+def test_e4m3_matches_torch_inside_the_range():
+    """torch's float8_e4m3fn cast (round to nearest even) on a dense sweep,
+    the subnormal range and exact midpoints; torch turns values past the
+    range into NaN, so the sweep stops below 464."""
+    import torch
+    g = np.random.Generator(np.random.PCG64(62))
+    x = np.concatenate([np.linspace(-463.9, 463.9, 100001), g.standard_normal(20000) * 1e-2,
+                        (np.arange(1, 64) + 0.5) * 2.0 ** -9])
+    ref = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_quantize(x, 1.0)
+    assert np.array_equal(oracle.e4m3_decode(got), oracle.e4m3_decode(ref))
+
+
+def test_e4m3_saturates_and_divides_by_the_scale():
+    assert list(oracle.e4m3_decode(oracle.e4m3_quantize([464.0, 1e6, -1e9, 500.0], 1.0))) == \
+        [448.0, 448.0, -448.0, 448.0]
+    x = np.linspace(-30, 30, 997)
+    assert np.array_equal(oracle.e4m3_quantize(x, 0.25), oracle.e4m3_quantize(x / 0.25, 1.0))
+
+
+# ---------------------------------------------------------------------------
 # Mutation tests: plant a mistake in the oracle; some pin must fail.
 # ---------------------------------------------------------------------------
 
@@ -488,3 +578,24 @@ def test_exp2_polynomial_constants_error_bound():
 
 ROOT_PTX = __import__("os").path.join(__import__("os").path.dirname(__import__("os").path.dirname(
     __import__("os").path.abspath(__file__))), "mla_prefill_attention_causal_b200", "csrc", "ptx.cuh")
+
+
+def test_mutant_sink_scaled_like_a_score(monkeypatch):
+    # the sink is already in score units: scaling it again must be caught
+    real = oracle.dense_prefill_sinks
+
+    def mutant(q, k, v, cu_q, cu_k, sc, causal, sinks, rows=None):
+        return real(q, k, v, cu_q, cu_k, sc, causal, np.asarray(sinks) * sc, rows=rows)
+    monkeypatch.setattr(oracle, "dense_prefill_sinks", mutant)
+    assert _fails_some_pin(SINK_PINS)
+
+
+def test_mutant_sink_left_out_of_the_lse(monkeypatch):
+    real = oracle.dense_prefill_sinks
+
+    def mutant(q, k, v, cu_q, cu_k, sc, causal, sinks, rows=None):
+        o, _ = real(q, k, v, cu_q, cu_k, sc, causal, sinks, rows=rows)
+        _, l = oracle.dense_prefill(q, k, v, cu_q, cu_k, sc, causal, rows=rows)
+        return o, l
+    monkeypatch.setattr(oracle, "dense_prefill_sinks", mutant)
+    assert _fails_some_pin(SINK_PINS)

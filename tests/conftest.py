@@ -19,3 +19,21 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionfinish(session, exitstatus):
+    mod = sys.modules.get("oracle_pool")
+    if mod is not None:
+        mod.close_pool()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the error figures of every whole-tensor oracle comparison."""
+    mod = sys.modules.get("oracle_pool")
+    if mod is None or not mod.SUMMARY:
+        return
+    terminalreporter.write_sep("-", "whole-tensor parity against the fp64 oracle")
+    for r in mod.SUMMARY:
+        terminalreporter.write_line(
+            f"{r['name']}: {r['values']} values, out max|err| {r['out_max']:.3g} "
+            f"mean {r['out_mean']:.3g}, lse max|err| {r['lse_max']:.3g}")

@@ -4,7 +4,7 @@ The kernel handles a token with two CTAs (value dims 0-255 and 256-511),
 64 selected rows per chunk, 128 heads as the MMA rows.  The cases cover a
 ragged last chunk, fewer heads than 128, -1 padding, out-of-range indices,
 a token with no valid index, duplicates, topk = 1, and the 4096-token
-workload (with and without padding) on sampled tokens.
+workload (with and without padding) on every token.
 """
 import numpy as np
 import pytest
@@ -16,6 +16,7 @@ import oracle
 pytestmark = pytest.mark.gpu
 
 from gpu_util import assert_lse_close, assert_out_close, dev_bf16, dev_i32, to_f64  # noqa: E402
+from oracle_pool import check_sparse_full  # noqa: E402
 
 
 def run_sparse(case, indices=None, want_lse=True):
@@ -125,9 +126,11 @@ def test_large_values_do_not_overflow(cuda_ok):
 
 
 @pytest.mark.parametrize("padded", [False, True])
-def test_workload_4096_tokens_sampled(cuda_ok, padded):
+def test_workload_4096_tokens_full(cuda_ok, padded):
+    """4096 tokens x 128 heads, top-k 2048 over a 32768-row cache: every
+    token and head against the oracle (padded: tokens at positions 0..4095,
+    so the first 2047 carry -1 fill)."""
     case = syn.sparse_config(seed=5, padded=padded)
-    g = np.random.Generator(np.random.PCG64(49))
-    tokens = sorted({0, 1, 63, 64, 2046, 2047, 2048, 4095} | set(int(x) for x in
-                                                                   g.integers(0, 4096, size=8)))
-    check_sparse(case, tokens=tokens)
+    out, lse = run_sparse(case)
+    check_sparse_full(f"sparse 4096 x 128, top-k 2048{' padded' if padded else ''}",
+                      case["q"], case["kv"], case["indices"], case["scale"], out, lse)

@@ -163,8 +163,10 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
  *     MLA_NOALLOC_SCRATCH_BYTES, i.e. ceil(total_q / 512) + batch <= 8160;
  *     larger calls return MLA_ERR_SCRATCH_TOO_SMALL and launch nothing.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first
- *     call before capturing work into a graph on that device.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for
+ *     that device's CUDA context; a context created anew (for example
+ *     after cudaDeviceReset) gets the lookup again on its first call.  Make
+ *     that first call before capturing work into a graph on that device.
  *   - All calls share the one array.  The kernels rewrite everything they
  *     read from it, so nothing needs clearing between calls, but two calls
  *     whose kernels can overlap on the GPU (different streams without an
@@ -220,6 +222,8 @@ int mla_attn_merge(const void* o_a, const float* lse_a, const void* o_b, const f
  *   lse        float32 [num_heads, num_tokens] or NULL.
  *   softmax_scale finite, > 0 (1/sqrt(576) for the absorbed shape).
  *   num_heads  1..128.
+ *   num_tokens 0 <= num_tokens < 2^30 and num_tokens * num_heads < 2^31
+ *              (otherwise MLA_ERR_INVALID_ARG, nothing launched).
  */
 int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* indices,
                            int topk, float softmax_scale, void* out, float* lse,

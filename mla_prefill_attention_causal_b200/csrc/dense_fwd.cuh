@@ -17,11 +17,19 @@
 // Work unit ("tile"): (sequence, 512-row query block, head) = two M=256
 // sub-tiles that share every K/V block.  A planner kernel sorts the
 // (sequence, query block) entries by their number of visible KV blocks,
-// longest first, into the caller's workspace; the persistent clusters walk
-// that list head-major in a static snake order (cluster c takes tile
-// k*C + c on even rounds and k*C + C-1-c on odd ones), so both CTAs of a
-// pair derive the same tile sequence without talking, clusters running at
-// the same time share K/V in L2, and the short tiles come last.
+// longest first, into the caller's workspace.  Tile t of the resulting list
+// is taken head-major (all entries of head 0, then of head 1, ...), except
+// for the last kTailHeads heads, which are taken entry-major (the longest
+// entry of each of those heads, then the next, ...): clusters running at
+// the same time then share the K/V of few heads in L2, and the list ends
+// with the shortest tiles of the call.  The persistent clusters take tiles
+// dynamically: cluster c starts with tile c, and whenever its producer warp
+// is ready for another tile it takes the next index from a counter in the
+// workspace, so a cluster that finishes early takes more work (greedy list
+// scheduling over a longest-first list).  The producer hands each tile's
+// coordinates to the other roles of both CTAs through a small ring in
+// shared memory.  Which cluster runs a tile does not change how the tile is
+// computed, so the output stays bitwise deterministic.
 //
 // Roles inside each CTA (384 threads):
 //   warps 0-3  softmax + epilogue, sub-tile 0 (thread = query row = TMEM lane)
@@ -83,22 +91,29 @@ static_assert(8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs <= kThreads * kLaunchR
 constexpr int kTmemCols = 512;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBins = 4096;                      // work histogram bins (clamped)
+constexpr int kTailHeads = 16;                       // heads taken entry-major at the end
+constexpr int kTileSlots = 4;                        // tiles in flight in the hand-off ring
 
 // Workspace layout (caller-provided device memory, 16-byte aligned).
 struct WsHeader {
   int num_entries;  // E: (sequence, 512-row block) entries
   int num_tiles;    // E * num_heads
-  int pad[2];
+  int next_tile;    // tiles taken from the counter so far (reset by the planner)
+  int pad;
 };
 constexpr size_t kWsHeaderBytes = 256;
 
-struct TileInfo {
+struct alignas(16) TileInfo {
   int q_start, Lq, k_start, Lk;
   int m0, h, valid, pad;
 };
 
-struct alignas(8) Bars {
-  uint64_t q_full[2];    // leader: Q bytes of both CTAs
+struct alignas(16) Bars {
+  TileInfo tiles[kTileSlots];     // both: tile hand-off ring (written by the leader's producer)
+  static_assert(sizeof(TileInfo) == 32, "a ring slot is two 16-byte stores");
+  uint64_t tile_full[kTileSlots];   // both: the slot holds the next tile
+  uint64_t tile_empty[kTileSlots];  // leader: every reader of the slot is done with it
+  uint64_t q_full[2];    // leader: both producers (and the Q bytes of both CTAs)
   uint64_t q_empty[2];   // both: last S MMA of the tile done
   uint64_t full_kv[kSlots];  // leader: K- and V-half bytes of block b, both CTAs
   uint64_t empty_k[kSlots];  // both: the S MMAs reading the K slot done
@@ -119,7 +134,7 @@ struct Params {
   const int* cu_k;
   __nv_bfloat16* out;
   float* lse;
-  const WsHeader* ws;
+  WsHeader* ws;
   const int2* entries;  // [E] {sequence, 512-row block index}, longest first
   int num_heads;
   int total_q;
@@ -214,6 +229,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int e = min(s_total, capacity);
     ws->num_entries = e;
     ws->num_tiles = e * num_heads;
+    ws->next_tile = 0;
   }
   __syncthreads();
   for (int b = tid; b < batch; b += blockDim.x) {
@@ -227,23 +243,35 @@ __global__ void __launch_bounds__(kPlanThreads)
   }
 }
 
-// Tile k of cluster c (static snake order over the sorted entry list).
-__device__ __forceinline__ TileInfo tile_at(const Params& p, int k, int cluster, int nclusters,
-                                            int num_tiles, int num_entries) {
-  const long long t = static_cast<long long>(k) * nclusters +
-                      ((k & 1) ? (nclusters - 1 - cluster) : cluster);
+// Coordinates of tile t of the list: head-major over the sorted entries,
+// then entry-major over the last kTailHeads heads (see the file comment).
+__device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_tiles,
+                                              int num_entries) {
   TileInfo ti;
   ti.valid = t < num_tiles ? 1 : 0;
+  ti.pad = 0;
   if (ti.valid) {
-    const int tt = static_cast<int>(t);
-    const int h = tt / num_entries;
-    const int2 e = p.entries[tt - h * num_entries];
-    ti.q_start = p.cu_q[e.x];
-    ti.Lq = p.cu_q[e.x + 1] - ti.q_start;
-    ti.k_start = p.cu_k[e.x];
-    ti.Lk = p.cu_k[e.x + 1] - ti.k_start;
-    ti.m0 = e.y * kTileRows;
+    const int H = p.num_heads;
+    const int tail = min(H, kTailHeads);
+    const int bulk = (H - tail) * num_entries;
+    int h, e;
+    if (t < bulk) {
+      h = t / num_entries;
+      e = t - h * num_entries;
+    } else {
+      const int u = t - bulk;
+      e = u / tail;
+      h = H - tail + (u - e * tail);
+    }
+    const int2 en = p.entries[e];
+    ti.q_start = p.cu_q[en.x];
+    ti.Lq = p.cu_q[en.x + 1] - ti.q_start;
+    ti.k_start = p.cu_k[en.x];
+    ti.Lk = p.cu_k[en.x + 1] - ti.k_start;
+    ti.m0 = en.y * kTileRows;
     ti.h = h;
+  } else {
+    ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.m0 = ti.h = 0;
   }
   return ti;
 }
@@ -289,7 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars->q_full[i]), 1);
+      // both producers arrive on every tile, with or without a Q load, so
+      // neither can fall behind the q_empty phase it waits for
+      mbar_init(smem_u32(&bars->q_full[i]), 2);
       mbar_init(smem_u32(&bars->q_empty[i]), 1);
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->p_full[i]), 8);
@@ -300,6 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->full_kv[i]), 1);
       mbar_init(smem_u32(&bars->empty_k[i]), 1);
       mbar_init(smem_u32(&bars->empty_v[i]), 1);
+    }
+    for (int i = 0; i < kTileSlots; ++i) {
+      mbar_init(smem_u32(&bars->tile_full[i]), 1);
+      // readers of a slot: the peer's producer, the MMA warp and the 16
+      // softmax warps of the pair
+      mbar_init(smem_u32(&bars->tile_empty[i]), 18);
     }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort = 0;
@@ -320,6 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
     return mbar_wait_cluster(bar, parity, abort_flag, err, tlim);
   };
+  // Slot and phase of the k-th tile in the hand-off ring.
+  auto tile_slot = [](int k) { return k % kTileSlots; };
+  auto tile_par = [](int k) { return static_cast<uint32_t>(k / kTileSlots) & 1u; };
 
   if (warp >= 8) {
     setmaxnreg_dec<kOtherRegs>();
@@ -334,7 +373,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       int blk = 0;  // KV blocks issued so far (slot = blk % kSlots)
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const TileInfo ti = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
+        // The leader takes the cluster's next tile and publishes it to both
+        // CTAs; the peer's producer reads its copy.
+        const int ts = tile_slot(k);
+        TileInfo ti;
+        if (leader) {
+          if (!(ok = wait(smem_u32(&bars->tile_empty[ts]), tile_par(k) ^ 1u,
+                          MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
+            break;
+          const int t = k == 0 ? cluster : nclusters + atomicAdd(&p.ws->next_tile, 1);
+          ti = tile_info(p, t, num_tiles, num_entries);
+          // Into both CTAs' slot: the barrier's phase completes once the
+          // 32 bytes have landed (st.async counts them on it).
+          const uint32_t a = smem_u32(&bars->tiles[ts]);
+          for (uint32_t r = 0; r < 2; ++r) {
+            const uint32_t fb = mapa_shared(smem_u32(&bars->tile_full[ts]), r);
+            mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(sizeof(TileInfo)));
+            st_async_v4(mapa_shared(a, r), ti.q_start, ti.Lq, ti.k_start, ti.Lk, fb);
+            st_async_v4(mapa_shared(a + 16, r), ti.m0, ti.h, ti.valid, ti.pad, fb);
+          }
+        } else {
+          if (!(ok = wait(smem_u32(&bars->tile_full[ts]), tile_par(k),
+                          MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
+            break;
+          ti = bars->tiles[ts];
+          if (ti.valid) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
+        }
         if (!ti.valid) break;
         int nb[2];
         tile_blocks(ti, causal, nb);
@@ -344,16 +408,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait(smem_u32(&bars->q_empty[i]), (static_cast<uint32_t>(k) & 1u) ^ 1u,
                           MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
+          // Both CTAs' producers arrive on the leader's q_full for every
+          // tile: the MMA warp then cannot finish with a tile's Q (and
+          // commit q_empty) before each producer has passed its q_empty
+          // wait for that tile.  Otherwise, for a sub-tile without rows
+          // (nothing to load), a late producer could find q_empty two
+          // phases on and wait on the wrong phase.
+          const uint32_t qbar = lead(&bars->q_full[i]);
           if (nb[i] > 0) {
-            if (leader) mbar_arrive_expect_tx(smem_u32(&bars->q_full[i]), 2 * kQSubBytes);
-            const uint32_t qbar = lead(&bars->q_full[i]);
+            if (leader)
+              mbar_arrive_expect_tx(smem_u32(&bars->q_full[i]), 2 * kQSubBytes);
+            else
+              mbar_arrive_cluster(qbar);
 #pragma unroll
             for (int c = 0; c < kQkChunks; ++c)
               tma_load_3d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q, 64 * c, ti.h,
                                ti.q_start + ti.m0 + i * kSubRows + static_cast<int>(rank) * kCtaRows,
                                qbar, pol_q);
-          } else if (leader) {
-            mbar_arrive(smem_u32(&bars->q_full[i]));
+          } else {
+            mbar_arrive_cluster(qbar);
           }
         }
         for (int n = 0; n < nblk && ok; ++n, ++blk) {
@@ -450,19 +523,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
+      // Tile k from the hand-off ring: whether it exists and the KV blocks
+      // of its two sub-tiles (read by every lane; lane 0 frees the slot).
+      auto fetch = [&](int k, int& valid, int (&n)[2]) -> bool {
+        const int ts = tile_slot(k);
+        if (!wait_bar(smem_u32(&bars->tile_full[ts]), tile_par(k))) return false;
+        const TileInfo ti = bars->tiles[ts];
+        __syncwarp();
+        if (ti.valid && lane == 0) mbar_arrive(smem_u32(&bars->tile_empty[ts]));
+        valid = ti.valid;
+        tile_blocks(ti, causal, n);
+        return true;
+      };
+
       int k = 0;
-      TileInfo cur = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
-      int nb[2];
-      tile_blocks(cur, causal, nb);
-      if (cur.valid) ok = start_tile(nb, blk, k);
-      while (ok && cur.valid) {
+      int cur_valid = 0, nxt_valid = 0;
+      int nb[2] = {0, 0}, nbn[2] = {0, 0};
+      ok = fetch(k, cur_valid, nb);
+      if (ok && cur_valid) ok = start_tile(nb, blk, k);
+      while (ok && cur_valid) {
         const int nblk = max(nb[0], nb[1]);
-        const TileInfo nxt = tile_at(p, k + 1, cluster, nclusters, num_tiles, num_entries);
-        int nbn[2];
-        tile_blocks(nxt, causal, nbn);
+        // The next tile is read when it is first needed (the last block of
+        // this one): the producer publishes it only after it has issued
+        // this tile's loads.
+        if (nblk == 0 && !(ok = fetch(k + 1, nxt_valid, nbn))) break;
         for (int n = 0; n < nblk && ok; ++n) {
           const int b = blk + n;  // this KV block; the next one is b + 1
           const bool last = n + 1 == nblk;
+          if (last && !(ok = fetch(k + 1, nxt_valid, nbn))) break;
           bool next_s[2] = {n + 1 < nb[0], n + 1 < nb[1]};
           if (last) {
             next_s[0] = nbn[0] > 0;
@@ -486,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             if (i == 1) commit_both(&bars->empty_v[b % kSlots]);  // V(b) no longer needed
-            if (last && nxt.valid &&
+            if (last && nxt_valid &&
                 !(ok = wait_bar(smem_u32(&bars->q_full[i]), static_cast<uint32_t>(k + 1) & 1u)))
               break;
             if (next_s[i]) {
@@ -495,17 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int nbi = last ? nbn[i] : nb[i];
               const int nidx = last ? 0 : n + 1;
               if (nidx == nbi - 1) commit_both(&bars->q_empty[i]);
-            } else if (last && nxt.valid) {
+            } else if (last && nxt_valid) {
               commit_both(&bars->q_empty[i]);  // no S for it in the next tile
             }
           }
           if (ok && more) commit_both(&bars->empty_k[(b + 1) % kSlots]);  // K(b+1) read by both S
         }
         if (!ok) break;
-        if (nblk == 0 && nxt.valid && !(ok = start_tile(nbn, blk, k + 1))) break;
+        if (nblk == 0 && nxt_valid && !(ok = start_tile(nbn, blk, k + 1))) break;
         blk += nblk;
         ++k;
-        cur = nxt;
+        cur_valid = nxt_valid;
         nb[0] = nbn[0];
         nb[1] = nbn[1];
       }
@@ -534,13 +622,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int o_cnt = 0;  // O-using tiles (o_full parity)
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const TileInfo ti = tile_at(p, k, cluster, nclusters, num_tiles, num_entries);
+      const int ts = tile_slot(k);
+      ok = __all_sync(0xffffffffu, wait(smem_u32(&bars->tile_full[ts]), tile_par(k),
+                                        MLA_DEVSTAT_WAIT_TIMEOUT_SOFTMAX));
+      if (!ok) break;
+      // The block loop needs only the row and key limits; the epilogue reads
+      // the tile's coordinates from the slot again (it stays valid until
+      // this warp frees it), which keeps them out of registers meanwhile.
+      const TileInfo ti = bars->tiles[ts];
       if (!ti.valid) break;
+      const int Lk = ti.Lk;
       const int row0 = ti.m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows;  // this CTA's rows
       const int r = row0 + wq * 32 + lane;  // row within the sequence
-      const int off = ti.Lk - ti.Lq;
-      const int nb = blocks_for(sub_tile_keys(ti.m0 + sub * kSubRows, ti.Lq, ti.Lk, causal));
-      const int lim = causal ? min(ti.Lk, r + off + 1) : ti.Lk;  // keys [0, lim) visible
+      const int off = Lk - ti.Lq;
+      const int nb = blocks_for(sub_tile_keys(ti.m0 + sub * kSubRows, ti.Lq, Lk, causal));
+      const int lim = causal ? min(Lk, r + off + 1) : Lk;  // keys [0, lim) visible
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
       float l_run = 0.f;        // running sum of the fp32 weights exp2(scaled s - m_run)
 
@@ -556,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(sraw[j]);
         const int kbase = n * kBlockKeys;
-        const bool full_blk = (kbase + kBlockKeys <= ti.Lk) &&
+        const bool full_blk = (kbase + kBlockKeys <= Lk) &&
                               (!causal || kbase + kBlockKeys - 1 <= row0 + off);
         if (!full_blk) {
 #pragma unroll
@@ -612,10 +708,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(pbar_lead);
       }
       if (!ok) break;
+      const int e_lq = bars->tiles[ts].Lq;
+      const int e_q0 = bars->tiles[ts].q_start;
+      const int e_h = bars->tiles[ts].h;
+      // Done with the tile's ring slot.  Freed here rather than at the start
+      // of the tile so that the cluster-scope release does not wait for the
+      // previous epilogue's stores.
+      __syncwarp();
+      if (lane == 0) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
 
       // ------------------------------------------------------- epilogue
-      const bool row_ok = r < ti.Lq;
-      const size_t row_index = static_cast<size_t>(ti.q_start + r) * p.num_heads + ti.h;
+      const bool row_ok = r < e_lq;
+      const size_t row_index = static_cast<size_t>(e_q0 + r) * p.num_heads + e_h;
       uint4* orow = reinterpret_cast<uint4*>(p.out + row_index * kDv);
       float lse_val = -INFINITY;
       if (nb > 0) {
@@ -651,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int v4 = 0; v4 < 16; ++v4) orow[v4] = make_uint4(0u, 0u, 0u, 0u);
       }
       if (row_ok && p.lse != nullptr)
-        p.lse[static_cast<size_t>(ti.h) * p.total_q + ti.q_start + r] = lse_val;
+        p.lse[static_cast<size_t>(e_h) * p.total_q + e_q0 + r] = lse_val;
     }
   }
 

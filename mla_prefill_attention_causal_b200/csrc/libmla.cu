@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -53,31 +54,57 @@ uint64_t wait_timeout_ns() {
   return t;
 }
 
-// Per-device one-time state: architecture check and kernel attributes.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context, or 0 when there is
+// none (or the driver cannot say).  A device's primary context is created
+// anew after cudaDeviceReset or after it was released, and what was set up
+// in the old one (kernel attributes, device addresses of module variables)
+// does not carry over, so the per-device state below is keyed on this id.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&c) != CUDA_SUCCESS || c == nullptr)
+    return 0;
+  unsigned long long id = 0;
+  return get_id(c, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// Per-device state, set up once per CUDA context: architecture check, kernel
+// attributes and launch sizes.  `ctx` is published last (release) and read
+// first (acquire), so a thread that sees its own context id there also sees
+// the fields written before it.
 struct DeviceState {
-  int checked = 0;  // 0 unknown, 1 ok, -1 unsupported
+  std::atomic<unsigned long long> ctx{0};  // context the fields belong to (0: none)
+  std::atomic<int> status{MLA_OK};         // MLA_OK or MLA_ERR_UNSUPPORTED
+  std::atomic<int> sms{0};
+  std::atomic<int> dense_clusters{0};      // co-resident 2-CTA clusters of the dense kernel
 };
 DeviceState g_dev[kMaxDevices];
-int g_dev_sms[kMaxDevices];
-int g_dev_dense_clusters[kMaxDevices];  // co-resident 2-CTA clusters of the dense kernel
 std::mutex g_dev_mu;
 
-int prepare_device(int* dev_out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
-  *dev_out = dev;
-  if (g_dev[dev].checked == 1) return MLA_OK;
-  if (g_dev[dev].checked == -1) return MLA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_dev_mu);
-  if (g_dev[dev].checked != 0) return g_dev[dev].checked == 1 ? MLA_OK : MLA_ERR_UNSUPPORTED;
+// The set-up itself (with the device's context current).
+int setup_device(int dev, int* status, int* sms, int* clusters) {
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (major != 10 || minor != 0) {
-    g_dev[dev].checked = -1;
-    return MLA_ERR_UNSUPPORTED;
+    *status = MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
   }
   if (cudaFuncSetAttribute(mla::dense::dense_fwd_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -90,8 +117,8 @@ int prepare_device(int* dev_out) {
     if (cudaFuncGetAttributes(&fa, mla::dense::dense_fwd_kernel) != cudaSuccess)
       return MLA_ERR_CUDA;
     if (fa.numRegs != mla::dense::kLaunchRegs) {
-      g_dev[dev].checked = -1;
-      return MLA_ERR_UNSUPPORTED;
+      *status = MLA_ERR_UNSUPPORTED;
+      return MLA_OK;
     }
   }
   if (cudaFuncSetAttribute(mla::sparse::sparse_fwd_kernel,
@@ -99,7 +126,7 @@ int prepare_device(int* dev_out) {
                            mla::sparse::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (encode_fn() == nullptr) return MLA_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MLA_ERR_CUDA;
   {
     cudaLaunchConfig_t cfg = {};
@@ -108,19 +135,48 @@ int prepare_device(int* dev_out) {
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2), 1, 1);
+    cfg.gridDim = dim3(2 * (*sms / 2), 1, 1);
     cfg.blockDim = dim3(mla::dense::kThreads, 1, 1);
     cfg.dynamicSmemBytes = mla::dense::kSmemBytes;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mla::dense::dense_fwd_kernel, &cfg) != cudaSuccess ||
-        n < 1)
+    if (cudaOccupancyMaxActiveClusters(clusters, mla::dense::dense_fwd_kernel, &cfg) !=
+            cudaSuccess ||
+        *clusters < 1)
       return MLA_ERR_CUDA;
-    g_dev_dense_clusters[dev] = n;
   }
-  g_dev[dev].checked = 1;
+  *status = MLA_OK;
   return MLA_OK;
+}
+
+// Checks the current device and sets it up in its current context (once per
+// context).  On success *dev_out is the device.
+int prepare_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  DeviceState& d = g_dev[dev];
+  unsigned long long ctx = current_context_id();
+  if (ctx != 0 && d.ctx.load(std::memory_order_acquire) == ctx)
+    return d.status.load(std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (ctx == 0) {
+    // No context is current yet: the runtime creates the device's primary
+    // context lazily; cudaSetDevice makes it current now.
+    if (cudaSetDevice(dev) != cudaSuccess) return MLA_ERR_CUDA;
+    ctx = current_context_id();
+  }
+  if (ctx != 0 && d.ctx.load(std::memory_order_relaxed) == ctx)
+    return d.status.load(std::memory_order_relaxed);
+  int status = MLA_OK, sms = 0, clusters = 0;
+  const int st = setup_device(dev, &status, &sms, &clusters);
+  if (st != MLA_OK) return st;
+  d.status.store(status, std::memory_order_relaxed);
+  d.sms.store(sms, std::memory_order_relaxed);
+  d.dense_clusters.store(clusters, std::memory_order_relaxed);
+  d.ctx.store(ctx, std::memory_order_release);  // 0 (unknown context): set up again next call
+  return status;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -166,25 +222,40 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ER
 
 // Scratch for mla_prefill_fwd_noalloc: the dense kernels' work list for
 // callers that cannot allocate.  In host code `g_noalloc_scratch` is only a
-// stand-in symbol; the device address comes from cudaGetSymbolAddress, once
-// per device (with that device current), and is cached here.
+// stand-in symbol; the device address comes from cudaGetSymbolAddress, with
+// the device current, once per device and CUDA context (a context created
+// anew, e.g. after cudaDeviceReset, may place the array elsewhere), and is
+// cached here.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
-void* g_noalloc_ptr[kMaxDevices];
+struct NoallocScratch {
+  std::atomic<unsigned long long> ctx{0};  // context `ptr` belongs to (0: none)
+  std::atomic<void*> ptr{nullptr};
+};
+NoallocScratch g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
+// Device address of the scratch array in the current context of `dev`
+// (prepare_device has made that context current).
 int noalloc_scratch(int dev, void** out) {
-  if (g_noalloc_ptr[dev] == nullptr) {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-        cudaGetLastError();
-        return MLA_ERR_CUDA;
-      }
-      g_noalloc_ptr[dev] = p;
-    }
+  NoallocScratch& n = g_noalloc[dev];
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && n.ctx.load(std::memory_order_acquire) == ctx) {
+    *out = n.ptr.load(std::memory_order_relaxed);
+    return MLA_OK;
   }
-  *out = g_noalloc_ptr[dev];
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (ctx != 0 && n.ctx.load(std::memory_order_relaxed) == ctx) {
+    *out = n.ptr.load(std::memory_order_relaxed);
+    return MLA_OK;
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  n.ptr.store(p, std::memory_order_relaxed);
+  n.ctx.store(ctx, std::memory_order_release);
+  *out = p;
   return MLA_OK;
 }
 
@@ -272,8 +343,10 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
     return MLA_ERR_INVALID_ARG;
   const size_t need = mla_prefill_workspace_size(batch, total_q);
   if (workspace_bytes < need) return MLA_ERR_INVALID_ARG;
-  // the kernels count tiles (work-list entries x heads) in int
-  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * num_heads > INT32_MAX)
+  // the kernels count tiles (work-list entries x heads, plus one grab per
+  // cluster past the end) in int
+  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * num_heads >
+      INT32_MAX - 65536)
     return MLA_ERR_INVALID_ARG;
   int dev = 0;
   int st = prepare_device(&dev);
@@ -313,8 +386,8 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
   // Persistent: as many 2-CTA clusters as can be resident at once, but never
   // more than tiles could exist.
   const long long max_tiles = static_cast<long long>(capacity) * num_heads;
-  const long long clusters =
-      max_tiles < g_dev_dense_clusters[dev] ? max_tiles : g_dev_dense_clusters[dev];
+  const long long resident = g_dev[dev].dense_clusters.load(std::memory_order_relaxed);
+  const long long clusters = max_tiles < resident ? max_tiles : resident;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -343,11 +416,10 @@ int mla_prefill_fwd_noalloc(const void* q, const void* k, const void* v,
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_SCRATCH_TOO_SMALL;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
-  void* scratch = nullptr;
-  const int st = noalloc_scratch(dev, &scratch);
+  int st = prepare_device(&dev);
   if (st != MLA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != MLA_OK) return st;
   return mla_prefill_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                          softmax_scale, causal, out, lse, stream, batch, num_heads, total_q,
                          total_k, scratch, MLA_NOALLOC_SCRATCH_BYTES);
@@ -371,8 +443,7 @@ int mla_attn_merge(const void* o_a, const float* lse_a, const void* o_b, const f
   const long long rows = static_cast<long long>(num_tokens) * num_heads;
   const int vpr = head_dim / 8;
   const long long vecs = rows * vpr;
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = g_dev[dev].sms.load(std::memory_order_relaxed);
   const long long want = (vecs + mla::merge::kThreads - 1) / mla::merge::kThreads;
   const long long cap = static_cast<long long>(sms) * 8;  // 8 resident CTAs of 256 per SM
   const int blocks = static_cast<int>(want < cap ? want : cap);
@@ -394,8 +465,9 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* 
   if (topk < 1 || num_tokens < 0 || num_heads < 1 || num_heads > 128 || num_kv_rows < 1)
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
-  // grid = 2 CTAs per token; TMA row coordinates are int32
-  if (num_tokens > (1 << 30) || static_cast<int64_t>(num_tokens) * num_heads > INT32_MAX)
+  // grid = 2 CTAs per token (an int); TMA row coordinates are int32
+  if (2 * static_cast<int64_t>(num_tokens) > INT32_MAX ||
+      static_cast<int64_t>(num_tokens) * num_heads > INT32_MAX)
     return MLA_ERR_INVALID_ARG;
   int dev = 0;
   int st = prepare_device(&dev);

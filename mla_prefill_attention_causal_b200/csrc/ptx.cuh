@@ -217,6 +217,34 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Arrive with cluster-scope release: the thread's earlier shared-memory
+// reads and writes, in either CTA of the cluster, are ordered before the
+// arrival for a thread that waits with cluster-scope acquire.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// Arrive on an mbarrier of any CTA of the cluster and add `bytes` to the
+// transaction count its current phase waits for.
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar,
+                                                              uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   cluster_bar),
+               "r"(bytes)
+               : "memory");
+}
+// Asynchronous 16-byte store into the shared memory of a CTA of the cluster,
+// counted as 16 bytes of transaction on that CTA's mbarrier `cluster_bar`:
+// a thread that sees the barrier's phase complete also sees the data (a
+// plain remote store followed by an arrive gives no such guarantee in
+// practice: the arrival can overtake the data).
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, int a, int b, int c, int d,
+                                            uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(cluster_addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
+      : "memory");
+}
 __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity,
                                                        bool suspend) {
   uint32_t ok;

@@ -100,6 +100,27 @@ def test_sparse_rejects_bad_arguments():
     assert f(None, P(16), P(16), 8, 0.1, P(16), None, None, 4, 128, 10) == _lib.MLA_ERR_INVALID_ARG
     assert f(P(16), P(16), P(16), 0, 0.1, P(16), None, None, 4, 128, 10) == _lib.MLA_ERR_INVALID_ARG
     assert f(P(16), P(16), P(16), 8, 0.1, P(16), None, None, 4, 129, 10) == _lib.MLA_ERR_INVALID_ARG
+    # two CTAs per token: 2^30 tokens would make a grid of 2^31 CTAs
+    assert f(P(16), P(16), P(16), 8, 0.1, P(16), None, None, 1 << 30, 1, 10) == \
+        _lib.MLA_ERR_INVALID_ARG
+
+
+def _call_noalloc(batch, total_q):
+    P = ctypes.c_void_p
+    return mla.load().mla_prefill_fwd_noalloc(P(16), P(16), P(16), P(16), P(16), 1, 1, 0.1, 1,
+                                              P(16), None, None, batch, 1, total_q, total_q)
+
+
+def test_noalloc_scratch_limit_at_its_edge():
+    """The fixed scratch holds ceil(total_q/512) + batch <= 8160 work-list
+    entries; one more is refused before the device is touched."""
+    assert mla.prefill_workspace_size(8144, 8144) == 65536       # 16 + 8144 = 8160 entries
+    assert mla.prefill_workspace_size(8145, 8145) == 65536 + 8   # 8161 entries
+    assert _call_noalloc(8145, 8145) == _lib.MLA_ERR_SCRATCH_TOO_SMALL
+    assert _call_noalloc(1, 8161 * 512) == _lib.MLA_ERR_SCRATCH_TOO_SMALL
+    # at the limit the size check passes (what follows needs a GPU)
+    assert _call_noalloc(8144, 8144) != _lib.MLA_ERR_SCRATCH_TOO_SMALL
+    assert "scratch" in _lib.status_string(_lib.MLA_ERR_SCRATCH_TOO_SMALL)
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch):

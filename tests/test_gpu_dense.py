@@ -10,6 +10,7 @@ pytestmark = pytest.mark.gpu
 
 from gpu_util import (assert_lse_close, assert_out_close, check_dense, dev_bf16, dev_i32,  # noqa: E402
                       run_dense, sample_rows, to_f64)
+from oracle_pool import check_dense_full  # noqa: E402
 
 
 @pytest.fixture(autouse=True)
@@ -73,6 +74,31 @@ def test_large_scores_rescale_the_running_max(causal):
     widened = (case["q"].astype(np.uint32) << np.uint32(16)).view(np.float32)
     case = dict(case, q=syn.f32_to_bf16_bits(widened * np.float32(32.0)))
     check_dense(case)
+
+
+def test_tile_handoff_across_alternating_launches():
+    """The persistent clusters hand each tile's coordinates from the leader
+    CTA to both CTAs through a ring in shared memory.  Alternating a call
+    whose clusters run several tiles with one whose clusters end after an
+    empty-key tile leaves different contents in the ring slots of the SMs;
+    a consumer that read a slot before its new contents landed would act on
+    the previous launch's tile (and give up waiting, or compute another
+    tile).  200 alternating calls: bitwise-stable outputs, no wait given up."""
+    import mla_prefill_attention_causal_b200 as mla
+    a = syn.dense_case([300, 1000, 129, 2000], [300, 1000, 129, 2000], 64, seed=21)
+    b = syn.dense_case([40, 70], [0, 90], 2, seed=14, causal=False)
+    ins = []
+    for c in (a, b):
+        ins.append((dev_bf16(c["q"]), dev_bf16(c["k"]), dev_bf16(c["v"]), dev_i32(c["cu_q"]),
+                    dev_i32(c["cu_k"]), c["max_q"], c["max_k"], c["scale"]))
+    ref = [mla.mla_prefill_fwd(*x, causal=c["causal"]) for x, c in zip(ins, (a, b))]
+    outs = [(torch.empty_like(o), torch.empty_like(l)) for o, l in ref]
+    for _ in range(100):
+        for x, c, (o, l) in zip(ins, (a, b), outs):
+            mla.mla_prefill_fwd(*x, causal=c["causal"], out=o, lse=l)
+    torch.cuda.synchronize()
+    for (ro, rl), (o, l) in zip(ref, outs):
+        assert torch.equal(ro, o) and torch.equal(rl, l)
 
 
 def test_lse_optional_and_out_identical():
@@ -149,10 +175,13 @@ def test_thousands_of_heads_on_tiny_sequences():
     check_dense(syn.dense_case(lens, lens, 4096, seed=19))
 
 
-def test_varlen16k_config_sampled():
-    """8 sequences, lengths U[512,4096], 128 heads: sampled rows, all heads."""
+def test_varlen16k_config_full():
+    """8 sequences, lengths U[512,4096] (15843 tokens), 128 heads, causal:
+    every query row and head against the oracle."""
     case = syn.varlen16k_config()
-    check_dense(case, rows=sample_rows(case["lens_q"], seed=2))
+    out, lse = run_dense(case)
+    check_dense_full("varlen16k (8 x U[512,4096], 128 heads, causal)", case["q"], case["k"],
+                     case["v"], case["cu_q"], case["cu_k"], case["scale"], True, out, lse)
 
 
 def test_long32k_config_sampled():
@@ -163,9 +192,14 @@ def test_long32k_config_sampled():
     check_dense(case, rows=sorted(set(rows)))
 
 
+# heads of the chunked workload checked on every row (0 and the last included)
+CHUNKED_HEADS = sorted(set(range(0, 128, 4)) | {127})
+
+
 def test_chunked_prefill_with_context_merge():
     """Prefix pass (unmasked, LSE) + self pass (causal) + merge equals one
-    bottom-right causal pass over [prefix, chunk] (sampled rows)."""
+    bottom-right causal pass over [prefix, chunk]: every query row of the
+    4 x 2048-token chunks, on 33 of the 128 heads."""
     import mla_prefill_attention_causal_b200 as mla
     d = syn.chunked_config()
     q = dev_bf16(d["q"])
@@ -176,15 +210,18 @@ def test_chunked_prefill_with_context_merge():
     o2, l2 = mla.mla_prefill_fwd(q, ks, vs, cq, cq, d["chunk"], d["chunk"], d["scale"], causal=True)
     om, lm = mla.mla_attn_merge(o1, l1, o2, l2)
     torch.cuda.synchronize()
-    B, C, P, H = d["batch"], d["chunk"], d["prefix"], d["num_heads"]
-    rows = sample_rows([C] * B, seed=4, per_seq=12)
-    # oracle: one causal call over the concatenated keys of each sequence
+    k_cat, v_cat, cu_cat = chunked_concat(d)
+    check_dense_full("chunked (4 x 2048 over 16384 prefix, prefix + self + merge, 33 heads)",
+                     d["q"], k_cat, v_cat, d["cu_q"], cu_cat, d["scale"], True, om, lm,
+                     heads=CHUNKED_HEADS, heads_per_job=1)
+
+
+def chunked_concat(d):
+    """Each sequence's prefix keys followed by its own chunk's keys: the key
+    set that one bottom-right causal call over [prefix, chunk] sees."""
+    B, C, P = d["batch"], d["chunk"], d["prefix"]
     k_cat = np.concatenate([np.concatenate([d["k_prefix"][b * P:(b + 1) * P],
                                             d["k_self"][b * C:(b + 1) * C]]) for b in range(B)])
     v_cat = np.concatenate([np.concatenate([d["v_prefix"][b * P:(b + 1) * P],
                                             d["v_self"][b * C:(b + 1) * C]]) for b in range(B)])
-    ref_o, ref_l = oracle.dense_prefill(d["q"], k_cat, v_cat, d["cu_q"],
-                                        syn.cu_seqlens([P + C] * B), d["scale"], True, rows=rows)
-    idx = torch.as_tensor(rows, device=om.device)
-    assert_out_close(to_f64(om.index_select(0, idx)), ref_o, "merged out")
-    assert_lse_close(lm.index_select(1, idx).cpu().numpy().astype(np.float64), ref_l, "merged lse")
+    return k_cat, v_cat, syn.cu_seqlens([P + C] * B)

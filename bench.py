@@ -8,24 +8,32 @@ causal, fp32 LSE.  Throughput counts causal-adjusted algorithmic FLOPs:
 2 * (192 + 128) * heads * (visible query-key pairs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--workload dense|sparse|sparse-padded]
+                  [--workload dense|long32k|chunked|sparse|sparse-padded]
 
-``--workload sparse`` times the absorbed top-k path instead: one
-``mla_sparse_prefill_fwd`` call over 4096 tokens x 128 heads (q dim 576),
-a 32768-row latent cache and top-k 2048 (``sparse-padded``: the same with
-the tokens at the start of the cache, so early lists carry -1 padding);
-FLOPs count 2 * (576 + 512) * heads per valid slot.
+``--workload long32k`` times one 32768-token causal sequence (128 heads);
+``--workload chunked`` times the chunked prefill with context (a non-causal
+prefix pass, a causal self pass and ``mla_attn_merge``; the merge is also
+event-timed on its own against the HBM roofline); ``--workload sparse``
+times the absorbed top-k path instead: one ``mla_sparse_prefill_fwd`` call
+over 4096 tokens x 128 heads (q dim 576), a 32768-row latent cache and
+top-k 2048 (``sparse-padded``: the same with the tokens at the start of the
+cache, so early lists carry -1 padding); FLOPs count 2 * (576 + 512) *
+heads per valid slot.
 
 Multi-GPU (torchrun): every rank runs its own independent batch of the
 same workload (weak scaling, no collective on the data path); the value is
 the sum of all ranks' FLOPs over the slowest rank's time.
 
-Timing: CUDA events on the launching stream; inputs (Q+K+V = 2.4 GB) are
-larger than the 126 MB L2, so nothing is flushed between steps.  The
-roofline fraction is given against the measured burst bf16 peak and, as
-``frac_of_sustained``, against the measured sustained one; the default 30
-timed calls match the burst measurement, while a few hundred back-to-back
-calls run under the power cap and land near the sustained figure.
+``--gpus N`` without torchrun starts N ranks itself (torch.distributed.run on
+127.0.0.1); under torchrun, ``--gpus`` must equal WORLD_SIZE.
+
+Timing: CUDA events on the launching stream; the inputs (Q+K+V = 2.08 GB for
+the dense workload) are larger than the 126 MB L2, so nothing is flushed
+between steps.  The roofline fraction is given against the measured burst
+bf16 peak and, as ``frac_of_sustained``, against the measured sustained one;
+the default 30 timed calls match the burst measurement, while a few hundred
+back-to-back calls run under the power cap and land near the sustained
+figure.
 """
 from __future__ import annotations
 
@@ -122,8 +130,14 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def make_workload(seed: int, heads: int = 128):
+LONG_WORKLOAD = ("long single-sequence causal MLA prefill: 1 sequence of 32768 tokens, 128 heads, "
+                 "qk 192 (128 nope + 64 rope) / v 128, bf16 N(0,1), scale 1/sqrt(192), fp32 LSE")
+
+
+def make_workload(seed: int, heads: int = 128, long: bool = False):
     import mla_synth as syn
+    if long:
+        return syn.long32k_config(seed=seed, num_heads=heads)
     return syn.varlen16k_config(seed=seed, num_heads=heads)
 
 
@@ -170,18 +184,21 @@ def recorded_traffic_for(profile: str, files):
 # ---------------------------------------------------------------------------
 
 class DenseWorkload:
-    """Dense varlen causal prefill (the headline metric's configuration)."""
+    """Dense varlen causal prefill (the headline metric's configuration), or
+    with ``long`` the single 32768-token sequence."""
 
-    name = "dense"
     metric = METRIC
     kernel = "mla::dense::dense_fwd_kernel"
     sources = ("dense_fwd.cuh", "ptx.cuh")
     profile = "dense_fwd_varlen16k.md"
 
-    def __init__(self, dev, seed, heads):
+    def __init__(self, dev, seed, heads, long=False):
         import torch
         import oracle
-        self.case = case = make_workload(seed, heads=heads)
+        self.long = long
+        self.name = "long32k" if long else "dense"
+        self.profile = "dense_fwd_long32k.md" if long else "dense_fwd_varlen16k.md"
+        self.case = case = make_workload(seed, heads=heads, long=long)
         self.H = H = case["num_heads"]
         self.flops = oracle.dense_flops(case["lens_q"], case["lens_k"], H, True)
         to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
@@ -210,17 +227,33 @@ class DenseWorkload:
 
     def config(self):
         c = self.case
-        return {"workload": WORKLOAD, "batch": len(c["lens_q"]), "total_tokens": self.T,
+        return {"workload": LONG_WORKLOAD if self.long else WORKLOAD, "batch": len(c["lens_q"]),
+                "total_tokens": self.T,
                 "heads": self.H, "seq_lens": c["lens_q"], "flops_per_step": self.flops,
                 "l2": "inputs larger than L2 (Q+K+V %.2f GB > 126 MB); no flush" %
                       ((self.q.numel() + self.k.numel() + self.v.numel()) * 2 / 1e9)}
 
-    data = "synthetic (seeded N(0,1) bf16, lengths U[512,4096])"
+    @property
+    def data(self):
+        return ("synthetic (seeded N(0,1) bf16, one 32768-token sequence)" if self.long else
+                "synthetic (seeded N(0,1) bf16, lengths U[512,4096])")
 
     def oracle_sample(self):
-        """The fp64 oracle on heads 0-5 of the workload (all query rows)."""
+        """The fp64 oracle on heads 0-5 of the workload (all query rows); for
+        the long sequence, 2048 evenly spaced query rows of heads 0-1."""
         import oracle
-        c, h = self.case, list(range(6))
+        c = self.case
+        if self.long:
+            rows = list(range(7, self.T, self.T // 2048))
+            h = [0, 1]
+            t0 = time.perf_counter()
+            oracle.dense_prefill(c["q"][:, h], c["k"][:, h], c["v"][:, h], c["cu_q"], c["cu_k"],
+                                 c["scale"], True, rows=rows)
+            dt = time.perf_counter() - t0
+            f = 2 * (192 + 128) * len(h) * sum(r + 1 for r in rows)
+            return f, dt, (f"{len(rows)} evenly spaced query rows of heads 0-1 of the 32768-token "
+                           f"sequence ({f:.3e} FLOPs in {dt:.1f} s)")
+        h = list(range(6))
         t0 = time.perf_counter()
         oracle.dense_prefill(c["q"][:, h], c["k"][:, h], c["v"][:, h], c["cu_q"], c["cu_k"],
                              c["scale"], True)
@@ -230,10 +263,18 @@ class DenseWorkload:
                        f"({f:.3e} FLOPs in {dt:.1f} s)")
 
     def reference_step(self, i):
-        """All query rows of sequence (i mod B) for head (i mod H) through the oracle."""
+        """All query rows of sequence (i mod B) for head (i mod H) through the
+        oracle; for the long sequence, 512 rows of head (i mod H)."""
         import oracle
         c = self.case
         B, H = len(c["lens_q"]), c["num_heads"]
+        if self.long:
+            h = i % H
+            rows = list(range(i % 64, self.T, self.T // 512))
+            t0 = time.perf_counter()
+            oracle.dense_prefill(c["q"][:, h:h + 1], c["k"][:, h:h + 1], c["v"][:, h:h + 1],
+                                 c["cu_q"], c["cu_k"], c["scale"], True, rows=rows)
+            return 2 * (192 + 128) * sum(r + 1 for r in rows), time.perf_counter() - t0
         b, h = i % B, i % H
         q0, q1 = int(c["cu_q"][b]), int(c["cu_q"][b + 1])
         k0, k1 = int(c["cu_k"][b]), int(c["cu_k"][b + 1])
@@ -242,7 +283,11 @@ class DenseWorkload:
                              c["v"][k0:k1, h:h + 1], [0, q1 - q0], [0, k1 - k0], c["scale"], True)
         return oracle.dense_flops([q1 - q0], [k1 - k0], 1, True), time.perf_counter() - t0
 
-    reference_sample = "step i = all query rows of sequence (i mod 8) for head (i mod 128)"
+    @property
+    def reference_sample(self):
+        return ("step i = 512 evenly spaced query rows (offset i mod 64) of head (i mod 128)"
+                if self.long else
+                "step i = all query rows of sequence (i mod 8) for head (i mod 128)")
 
 
 class SparseWorkload:
@@ -449,6 +494,8 @@ def whole_job_value(flops_per_rank: float, world: int, ms_step: float) -> float:
 def make(args, dev, rank, world):
     if args.workload == "dense":
         return DenseWorkload(dev, rank_seed(2, rank, world), args.heads)
+    if args.workload == "long32k":
+        return DenseWorkload(dev, rank_seed(3, rank, world), args.heads, long=True)
     if args.workload == "chunked":
         return ChunkedWorkload(dev, rank_seed(4, rank, world), args.heads)
     return SparseWorkload(dev, rank_seed(5, rank, world), args.heads,
@@ -459,10 +506,11 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
     # The reference arm runs the oracle on the host only: build the host-side case.
-    if args.workload == "dense":
+    if args.workload in ("dense", "long32k"):
         w = DenseWorkload.__new__(DenseWorkload)
-        w.case = make_workload(2)
-        w.H = w.case["num_heads"]
+        w.long = args.workload == "long32k"
+        w.case = make_workload(3 if w.long else 2, long=w.long)
+        w.H, w.T = w.case["num_heads"], w.case["q"].shape[0]
     elif args.workload == "chunked":
         import mla_synth as syn
         w = ChunkedWorkload.__new__(ChunkedWorkload)
@@ -488,7 +536,8 @@ def run_reference(args, rank: int, world: int):
         "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": WORKLOAD if args.workload == "dense" else args.workload,
+        "config": {"workload": {"dense": WORKLOAD, "long32k": LONG_WORKLOAD}.get(args.workload,
+                                                                                  args.workload),
                    "sample": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
@@ -609,6 +658,18 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     return 0
 
 
+def relaunch_with_ranks(n: int) -> int:
+    """Start n ranks of this script (one per GPU) with torch.distributed.run."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -623,13 +684,22 @@ def main():
                     help="time the kernel only (no e2e, clocks or CPU baseline); for profiling")
     ap.add_argument("--heads", type=int, default=128,
                     help="heads of the dense workload (128 for the bench line; fewer for profiling)")
-    ap.add_argument("--workload", default="dense", choices=["dense", "chunked", "sparse", "sparse-padded"],
-                    help="dense: the headline configuration; chunked: prefix + self passes and "
-                         "the LSE merge; sparse: the absorbed top-k path")
+    ap.add_argument("--workload", default="dense",
+                    choices=["dense", "long32k", "chunked", "sparse", "sparse-padded"],
+                    help="dense: the headline configuration; long32k: one 32768-token causal "
+                         "sequence; chunked: prefix + self passes and the LSE merge; sparse: the "
+                         "absorbed top-k path")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch_with_ranks(args.gpus)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE is {world}", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if world > 1:

@@ -62,3 +62,28 @@ def test_single_rank_needs_no_process_group():
 def test_whole_job_value_is_weak_scaling_sum(world):
     # every rank did 1.5e12 FLOPs in (at most) 1.5 ms: 1000 TFLOP/s per rank
     assert bench.whole_job_value(1.5e12, world, 1.5) == pytest.approx(1000.0 * world)
+
+
+def test_gpus_flag_must_match_the_launched_world_size():
+    """Under torchrun the rank count comes from WORLD_SIZE; a --gpus that
+    disagrees is an error (exit 2) before any GPU work, not a silent 1-GPU run."""
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--steps", "1"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2, (r.returncode, r.stderr[-500:])
+    assert "WORLD_SIZE is 1" in r.stderr
+
+
+def test_gpus_flag_without_torchrun_starts_that_many_ranks(monkeypatch):
+    """--gpus N > 1 outside torchrun re-runs the script under
+    torch.distributed.run with N processes on 127.0.0.1."""
+    import subprocess
+    seen = {}
+    monkeypatch.setattr(subprocess, "call", lambda cmd: seen.setdefault("cmd", cmd) and 0)
+    assert bench.relaunch_with_ranks(4) == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"

@@ -8,12 +8,14 @@ causal, fp32 LSE.  Throughput counts causal-adjusted algorithmic FLOPs:
 2 * (192 + 128) * heads * (visible query-key pairs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--workload dense|long32k|chunked|sparse|sparse-padded]
+                  [--workload dense|long32k|chunked|chunked-context|sparse|sparse-padded]
 
 ``--workload long32k`` times one 32768-token causal sequence (128 heads);
 ``--workload chunked`` times the chunked prefill with context (a non-causal
 prefix pass, a causal self pass and ``mla_attn_merge``; the merge is also
-event-timed on its own against the HBM roofline); ``--workload sparse``
+event-timed on its own against the HBM roofline), ``--workload
+chunked-context`` the same in one ``mla_prefill_fwd_context`` call;
+``--workload sparse``
 times the absorbed top-k path instead: one ``mla_sparse_prefill_fwd`` call
 over 4096 tokens x 128 heads (q dim 576), a 32768-row latent cache and
 top-k 2048 (``sparse-padded``: the same with the tokens at the start of the
@@ -470,6 +472,39 @@ class ChunkedWorkload:
         return self._oracle_head(i % self.case["batch"], i % self.H)
 
 
+class ChunkedContextWorkload(ChunkedWorkload):
+    """The chunked workload in one pass: ``mla_prefill_fwd_context`` attends
+    to the prefix (every key) and to the chunk itself (causal) under one
+    softmax -- no partial outputs and no merge."""
+
+    name = "chunked-context"
+    metric = ("MLA chunked prefill in one pass (context + causal self keys) attn TFLOPS "
+              "(causal-adj) and % of B200 dense BF16 peak, 1 GPU")
+    profile = "dense_fwd_chunked_context.md"
+    reference_sample = ("step i = head (i mod 128) of sequence (i mod 4): prefix pass, self pass "
+                        "and merge of that head's 2048 query rows (the oracle's form of the "
+                        "one-pass result)")
+
+    def __init__(self, dev, seed, heads):
+        super().__init__(dev, seed, heads)
+        self.launches = 2  # planner + attention
+        self.merge_events = None
+
+    def step(self):
+        import mla_prefill_attention_causal_b200 as mla
+        c = self.case
+        mla.mla_prefill_fwd_context(self.q, self.ks, self.vs, self.cu_q, self.cu_q, self.kp,
+                                    self.vp, self.cu_p, c["chunk"], c["chunk"], c["prefix"],
+                                    c["scale"], causal=True, out=self.out, lse=self.lse)
+
+    def config(self):
+        cfg = super().config()
+        cfg["workload"] = cfg["workload"].replace("merged with mla_attn_merge",
+                                                  "in one pass (mla_prefill_fwd_context)")
+        cfg.pop("merge_bytes_per_step", None)
+        return cfg
+
+
 def rank_seed(base: int, rank: int, world: int) -> int:
     """Seed of a rank's batch: the workload's own seed on one GPU, and a
     distinct batch per rank under weak scaling."""
@@ -498,6 +533,8 @@ def make(args, dev, rank, world):
         return DenseWorkload(dev, rank_seed(3, rank, world), args.heads, long=True)
     if args.workload == "chunked":
         return ChunkedWorkload(dev, rank_seed(4, rank, world), args.heads)
+    if args.workload == "chunked-context":
+        return ChunkedContextWorkload(dev, rank_seed(4, rank, world), args.heads)
     return SparseWorkload(dev, rank_seed(5, rank, world), args.heads,
                           padded=args.workload == "sparse-padded")
 
@@ -511,9 +548,10 @@ def run_reference(args, rank: int, world: int):
         w.long = args.workload == "long32k"
         w.case = make_workload(3 if w.long else 2, long=w.long)
         w.H, w.T = w.case["num_heads"], w.case["q"].shape[0]
-    elif args.workload == "chunked":
+    elif args.workload in ("chunked", "chunked-context"):
         import mla_synth as syn
-        w = ChunkedWorkload.__new__(ChunkedWorkload)
+        cls = ChunkedWorkload if args.workload == "chunked" else ChunkedContextWorkload
+        w = cls.__new__(cls)
         w.case = syn.chunked_config(seed=4)
         w.H = w.case["num_heads"]
     else:
@@ -685,10 +723,11 @@ def main():
     ap.add_argument("--heads", type=int, default=128,
                     help="heads of the dense workload (128 for the bench line; fewer for profiling)")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "long32k", "chunked", "sparse", "sparse-padded"],
+                    choices=["dense", "long32k", "chunked", "chunked-context", "sparse",
+                             "sparse-padded"],
                     help="dense: the headline configuration; long32k: one 32768-token causal "
-                         "sequence; chunked: prefix + self passes and the LSE merge; sparse: the "
-                         "absorbed top-k path")
+                         "sequence; chunked: prefix + self passes and the LSE merge; "
+                         "chunked-context: the same in one pass; sparse: the absorbed top-k path")
     args = ap.parse_args()
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")

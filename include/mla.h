@@ -146,6 +146,66 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
                             int total_q, int total_k, void* workspace, size_t workspace_bytes);
 
 /*
+ * Chunked prefill in one pass.  For each sequence b, the queries attend to
+ * every key of its context (k_ctx / v_ctx rows [cu_seqlens_ctx[b],
+ * cu_seqlens_ctx[b+1]), no mask) and to its own keys (k / v rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]), with the causal mask of
+ * mla_prefill_fwd when causal == 1), under one softmax.  The result (out,
+ * and the LSE over both key sets) is what mla_attn_merge gives for a
+ * context pass (mla_prefill_fwd over the context, causal = 0, LSE
+ * returned) and a pass over the sequence's own keys -- the two passes of
+ * vLLM's MLA prefill backend ("flash_attn.py", run_prefill_context_chunk:
+ * unmasked, LSE returned; run_prefill_new_tokens: causal), merged by their
+ * LSEs -- without the partial outputs, the merge launch or their trip
+ * through HBM.  The kernel visits a tile's context blocks first, then its
+ * own visible blocks.
+ *   k_ctx        bf16 [total_ctx, num_heads, 192], packed, 16-B aligned.
+ *   v_ctx        bf16 [total_ctx, num_heads, 128], packed, 16-B aligned.
+ *   cu_seqlens_ctx int32 [batch + 1] on the device: cu[0] = 0,
+ *                non-decreasing, cu[batch] = total_ctx; a sequence may have
+ *                an empty context (the call is then mla_prefill_fwd for it).
+ *   max_seqlen_ctx, total_ctx  sizes (>= 0).
+ * Every other argument is that of mla_prefill_fwd (packed q, k, v; the same
+ * workspace size).  Returns MLA_OK or an error; on error nothing was
+ * launched.
+ */
+int mla_prefill_fwd_context(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            const void* k_ctx, const void* v_ctx, const int32_t* cu_seqlens_ctx,
+                            int max_seqlen_q, int max_seqlen_k, int max_seqlen_ctx,
+                            float softmax_scale, int causal, void* out, float* lse,
+                            mla_stream_t stream, int batch, int num_heads, int total_q,
+                            int total_k, int total_ctx, void* workspace, size_t workspace_bytes);
+
+/*
+ * mla_prefill_fwd with two options: attention sinks (the "Sgl project
+ * Sglang FA4 Interface" page, Description: learnable sink tokens; the
+ * SparseFlashMla README's `sinks` parameter; the Mojo sparse branch's
+ * attn_sink_ptr) and a static FP8 output scale (vLLM "flash_attn.py",
+ * supports_quant_output: kFp8StaticTensorSym, output_scale).
+ *   sinks         float [num_heads] device array, or NULL.  Head h's sink
+ *                 logit s_h (in the units of softmax_scale * q.k) joins
+ *                 every row's softmax with a zero value:
+ *                 O = sum_j e^x_j v_j / (e^s_h + sum_j e^x_j),
+ *                 LSE = ln(e^s_h + sum_j e^x_j); a row that sees no key gets
+ *                 O = 0 and LSE = s_h.  (The pages name the input, not its
+ *                 arithmetic; this is the plain reading of a sink token.)
+ *   output_scale  float device scalar, or NULL.  When set, `out` is e4m3
+ *                 (1 byte per element, [total_q, num_heads, 128], 16-B
+ *                 aligned) holding O / *output_scale rounded to nearest even
+ *                 and saturated at +-448; otherwise `out` is bf16 as in
+ *                 mla_prefill_fwd.
+ * Every other argument is that of mla_prefill_fwd (packed q, k, v).  With
+ * both options NULL the result is bit for bit that of mla_prefill_fwd.
+ */
+int mla_prefill_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                       const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+                       float softmax_scale, int causal, const float* sinks,
+                       const float* output_scale, void* out, float* lse, mla_stream_t stream,
+                       int batch, int num_heads, int total_q, int total_k, void* workspace,
+                       size_t workspace_bytes);
+
+/*
  * mla_prefill_fwd for callers that cannot allocate device memory.
  *
  * (The pages have no counterpart to this entry point; it is a convenience of

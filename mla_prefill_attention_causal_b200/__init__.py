@@ -12,6 +12,8 @@ from ._lib import (  # noqa: F401
     mla_debug_wait_timeout,
     mla_device_status,
     mla_prefill_fwd,
+    mla_prefill_fwd_context,
+    mla_prefill_fwd_ex,
     mla_sparse_prefill_fwd,
     prefill_workspace_size,
     status_string,

@@ -42,6 +42,10 @@ SIGNATURES = {
                              _S]),
     "mla_prefill_fwd_strided": (_I, [_P, _L, _L, _P, _L, _L, _P, _L, _L, _P, _P, _I, _I, _F, _I,
                                      _P, _P, _P, _I, _I, _I, _I, _P, _S]),
+    "mla_prefill_fwd_context": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _I, _P, _P,
+                                     _P, _I, _I, _I, _I, _I, _P, _S]),
+    "mla_prefill_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _P, _P, _I, _I, _I,
+                                _I, _P, _S]),
     "mla_prefill_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I,
                                      _I]),
     "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
@@ -188,6 +192,123 @@ def _prefill_call(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_
         st = load().mla_prefill_fwd_strided(_ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0),
                                             k.stride(1), _ptr(v), v.stride(0), v.stride(1), *rest)
         _check("mla_prefill_fwd_strided", st)
+    return out, lse
+
+
+def _packed_dense_args(q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale, out, lse,
+                       return_lse, workspace, out_dtype=torch.bfloat16):
+    """Checks shared by the packed dense calls; allocates what is missing."""
+    for t, n, d in ((q, "q", QK_DIM), (k, "k", QK_DIM), (v, "v", V_DIM)):
+        _need(t, n, torch.bfloat16, 3)
+        if t.shape[2] != d:
+            raise ValueError(f"{n} must be [*, H, {d}], got {tuple(t.shape)}")
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, num_heads, _ = q.shape
+    total_k = k.shape[0]
+    if k.shape[1] != num_heads or v.shape[:2] != (total_k, num_heads):
+        raise ValueError("q, k and v must agree on heads, k and v on rows")
+    batch = cu_seqlens_q.numel() - 1
+    if batch < 1 or cu_seqlens_k.numel() != batch + 1:
+        raise ValueError("cu_seqlens_q/k must both have batch+1 >= 2 entries")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(QK_DIM)
+    if out is None:
+        out = torch.empty((total_q, num_heads, V_DIM), dtype=out_dtype, device=q.device)
+    else:
+        _need(out, "out", out_dtype, 3)
+        if out.shape != (total_q, num_heads, V_DIM):
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((num_heads, total_q), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+        if lse.shape != (num_heads, total_q):
+            raise ValueError("lse must be [num_heads, total_q]")
+    ws_bytes = prefill_workspace_size(batch, total_q)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < ws_bytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of >= {ws_bytes} bytes")
+    return (float(softmax_scale), out, lse, workspace, batch, num_heads, total_q, total_k)
+
+
+def mla_prefill_fwd_context(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                            k_ctx: torch.Tensor, v_ctx: torch.Tensor, cu_seqlens_ctx: torch.Tensor,
+                            max_seqlen_q: int, max_seqlen_k: int, max_seqlen_ctx: int,
+                            softmax_scale: Optional[float] = None, causal: bool = True,
+                            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            return_lse: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Chunked prefill in one pass (``mla_prefill_fwd_context`` in ``mla.h``).
+
+    The queries attend to all of their sequence's context keys (``k_ctx`` /
+    ``v_ctx`` rows given by ``cu_seqlens_ctx``) and to their own keys (``k``
+    / ``v``, causal when ``causal``) under one softmax: the merged result of
+    a context pass and a new-token pass.  All tensors packed, bf16
+    ``[*, H, 192]`` / ``[*, H, 128]``; cu_seqlens int32 ``[B+1]``.
+    Returns ``(out [total_q, H, 128] bf16, lse [H, total_q] fp32 or None)``.
+    """
+    scale, out, lse, workspace, batch, num_heads, total_q, total_k = _packed_dense_args(
+        q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale, out, lse, return_lse, workspace)
+    for t, n, d in ((k_ctx, "k_ctx", QK_DIM), (v_ctx, "v_ctx", V_DIM)):
+        _need(t, n, torch.bfloat16, 3)
+        if t.shape[1:] != (num_heads, d):
+            raise ValueError(f"{n} must be [*, {num_heads}, {d}], got {tuple(t.shape)}")
+    _need(cu_seqlens_ctx, "cu_seqlens_ctx", torch.int32, 1)
+    total_ctx = k_ctx.shape[0]
+    if v_ctx.shape[0] != total_ctx or cu_seqlens_ctx.numel() != batch + 1:
+        raise ValueError("k_ctx / v_ctx rows or cu_seqlens_ctx entries do not match")
+    _same_device(q, k=k, v=v, k_ctx=k_ctx, v_ctx=v_ctx, cu_seqlens_q=cu_seqlens_q,
+                 cu_seqlens_k=cu_seqlens_k, cu_seqlens_ctx=cu_seqlens_ctx, out=out, lse=lse,
+                 workspace=workspace)
+    with torch.cuda.device(q.device):
+        st = load().mla_prefill_fwd_context(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(k_ctx),
+            _ptr(v_ctx), _ptr(cu_seqlens_ctx), int(max_seqlen_q), int(max_seqlen_k),
+            int(max_seqlen_ctx), scale, 1 if causal else 0, _ptr(out), _ptr(lse), _stream(),
+            batch, num_heads, total_q, total_k, total_ctx, _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    _check("mla_prefill_fwd_context", st)
+    return out, lse
+
+
+def mla_prefill_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                       max_seqlen_q: int, max_seqlen_k: int,
+                       softmax_scale: Optional[float] = None, causal: bool = True,
+                       sinks: Optional[torch.Tensor] = None,
+                       output_scale: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       return_lse: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Dense prefill with attention sinks and/or an FP8 output (``mla_prefill_fwd_ex``).
+
+    ``sinks``: float32 ``[H]`` (one logit per head) or None.  ``output_scale``:
+    a float32 one-element CUDA tensor or None; when given, ``out`` is
+    ``torch.float8_e4m3fn`` holding O / scale (round to nearest even,
+    saturated at 448).  Returns ``(out, lse)``.
+    """
+    fp8 = output_scale is not None
+    scale, out, lse, workspace, batch, num_heads, total_q, total_k = _packed_dense_args(
+        q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale, out, lse, return_lse, workspace,
+        out_dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
+    if sinks is not None:
+        _need(sinks, "sinks", torch.float32, 1)
+        if sinks.numel() != num_heads:
+            raise ValueError("sinks must hold one value per head")
+    if fp8:
+        _need(output_scale, "output_scale", torch.float32, 1)
+        if output_scale.numel() != 1:
+            raise ValueError("output_scale must be a one-element tensor")
+    _same_device(q, k=k, v=v, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, sinks=sinks,
+                 output_scale=output_scale, out=out, lse=lse, workspace=workspace)
+    with torch.cuda.device(q.device):
+        st = load().mla_prefill_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+            int(max_seqlen_k), scale, 1 if causal else 0, _ptr(sinks), _ptr(output_scale),
+            _ptr(out), _ptr(lse), _stream(), batch, num_heads, total_q, total_k, _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    _check("mla_prefill_fwd_ex", st)
     return out, lse
 
 

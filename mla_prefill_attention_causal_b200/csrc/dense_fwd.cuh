@@ -19,10 +19,11 @@
 // (sequence, query block) entries by their number of visible KV blocks,
 // longest first, into the caller's workspace.  Tile t of the resulting list
 // is taken head-major (all entries of head 0, then of head 1, ...), except
-// for the last kTailHeads heads, which are taken entry-major (the longest
-// entry of each of those heads, then the next, ...): clusters running at
-// the same time then share the K/V of few heads in L2, and the list ends
-// with the shortest tiles of the call.  The persistent clusters take tiles
+// for the last few heads -- enough for about three rounds of the clusters
+// -- which are taken entry-major (the longest entry of each of those
+// heads, then the next, ...): clusters running at the same time then share
+// the K/V of few heads in L2, and the list ends with the shortest tiles of
+// the call.  The persistent clusters take tiles
 // dynamically: cluster c starts with tile c, and whenever its producer warp
 // is ready for another tile it takes the next index from a counter in the
 // workspace, so a cluster that finishes early takes more work (greedy list
@@ -91,7 +92,7 @@ static_assert(8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs <= kThreads * kLaunchR
 constexpr int kTmemCols = 512;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBins = 4096;                      // work histogram bins (clamped)
-constexpr int kTailHeads = 16;                       // heads taken entry-major at the end
+constexpr int kTailRounds = 3;                       // rounds of clusters the entry-major tail spans
 constexpr int kTileSlots = 4;                        // tiles in flight in the hand-off ring
 
 // Workspace layout (caller-provided device memory, 16-byte aligned).
@@ -103,9 +104,14 @@ struct WsHeader {
 };
 constexpr size_t kWsHeaderBytes = 256;
 
+// A tile: its sequence's queries, keys and (for a call with a context, see
+// mla_prefill_fwd_context) context keys, the first query row and the head.
+// A tile always has query rows, so Lq == 0 marks "no tile" (the end of a
+// cluster's list).
 struct alignas(16) TileInfo {
   int q_start, Lq, k_start, Lk;
-  int m0, h, valid, pad;
+  int c_start, Lc, m0, h;
+  __host__ __device__ bool valid() const { return Lq > 0; }
 };
 
 struct alignas(16) Bars {
@@ -132,8 +138,11 @@ constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + static_cast<int>(sizeof
 struct Params {
   const int* cu_q;
   const int* cu_k;
-  __nv_bfloat16* out;
+  const int* cu_ctx;       // context keys per sequence ([batch + 1]), or null: no context
+  void* out;               // bf16 [total_q, H, 128], or e4m3 when out_scale is set
   float* lse;
+  const float* sinks;      // one attention-sink logit per head, or null
+  const float* out_scale;  // e4m3 output scale (device scalar), or null: bf16 output
   WsHeader* ws;
   const int2* entries;  // [E] {sequence, 512-row block index}, longest first
   int num_heads;
@@ -157,31 +166,41 @@ __host__ __device__ __forceinline__ int sub_tile_keys(int row0, int Lq, int Lk, 
 __host__ __device__ __forceinline__ int blocks_for(int keys) {
   return (keys + kBlockKeys - 1) / kBlockKeys;
 }
+// KV blocks a 256-row sub-tile starting at row0 visits: every block of the
+// sequence's context first (all context keys are visible), then the blocks
+// of its own visible keys; none when it has no rows.
+__host__ __device__ __forceinline__ int sub_tile_blocks(int row0, int Lq, int Lk, int Lc,
+                                                        int causal) {
+  if (row0 >= Lq) return 0;
+  return blocks_for(Lc) + blocks_for(sub_tile_keys(row0, Lq, Lk, causal));
+}
 
 // ------------------------------------------------------------------ planner
 // One CTA: builds the (sequence, 512-row block) entry list sorted by the
 // number of KV blocks its rows visit (descending).
 __global__ void __launch_bounds__(kPlanThreads)
-    dense_plan_kernel(const int* cu_q, const int* cu_k, int batch, int causal, WsHeader* ws,
-                      int2* entries, int capacity, int num_heads) {
+    dense_plan_kernel(const int* cu_q, const int* cu_k, const int* cu_ctx, int batch,
+                      int causal, WsHeader* ws, int2* entries, int capacity, int num_heads) {
   __shared__ int bins[kPlanBins];
   __shared__ int s_total;
   const int tid = threadIdx.x;
   for (int i = tid; i < kPlanBins; i += blockDim.x) bins[i] = 0;
   if (tid == 0) s_total = 0;
   __syncthreads();
-  auto work_of = [&](int Lq, int Lk, int mb) -> int {
+  auto work_of = [&](int Lq, int Lk, int Lc, int mb) -> int {
     const int m0 = mb * kTileRows;
-    const int k0 = sub_tile_keys(m0, Lq, Lk, causal);
-    const int k1 = sub_tile_keys(m0 + kSubRows, Lq, Lk, causal);
-    return min(kPlanBins - 1, blocks_for(max(k0, k1)));
+    const int n0 = sub_tile_blocks(m0, Lq, Lk, Lc, causal);
+    const int n1 = sub_tile_blocks(m0 + kSubRows, Lq, Lk, Lc, causal);
+    return min(kPlanBins - 1, max(n0, n1));
   };
+  auto ctx_of = [&](int b) -> int { return cu_ctx != nullptr ? cu_ctx[b + 1] - cu_ctx[b] : 0; };
   for (int b = tid; b < batch; b += blockDim.x) {
     const int Lq = cu_q[b + 1] - cu_q[b];
     const int Lk = cu_k[b + 1] - cu_k[b];
+    const int Lc = ctx_of(b);
     const int nmb = (Lq + kTileRows - 1) / kTileRows;
     atomicAdd(&s_total, nmb);
-    for (int mb = 0; mb < nmb; ++mb) atomicAdd(&bins[work_of(Lq, Lk, mb)], 1);
+    for (int mb = 0; mb < nmb; ++mb) atomicAdd(&bins[work_of(Lq, Lk, Lc, mb)], 1);
   }
   __syncthreads();
   {
@@ -235,24 +254,29 @@ __global__ void __launch_bounds__(kPlanThreads)
   for (int b = tid; b < batch; b += blockDim.x) {
     const int Lq = cu_q[b + 1] - cu_q[b];
     const int Lk = cu_k[b + 1] - cu_k[b];
+    const int Lc = ctx_of(b);
     const int nmb = (Lq + kTileRows - 1) / kTileRows;
     for (int mb = nmb - 1; mb >= 0; --mb) {
-      const int pos = atomicAdd(&bins[work_of(Lq, Lk, mb)], 1);
+      const int pos = atomicAdd(&bins[work_of(Lq, Lk, Lc, mb)], 1);
       if (pos < capacity) entries[pos] = make_int2(b, mb);
     }
   }
 }
 
+// Heads taken entry-major at the end of the list: enough for kTailRounds
+// rounds of the clusters, at least one.
+__device__ __forceinline__ int tail_heads(int num_heads, int num_entries, int nclusters) {
+  const int want = (kTailRounds * nclusters + num_entries - 1) / max(num_entries, 1);
+  return max(1, min(num_heads, want));
+}
+
 // Coordinates of tile t of the list: head-major over the sorted entries,
-// then entry-major over the last kTailHeads heads (see the file comment).
+// then entry-major over the last `tail` heads (see the file comment).
 __device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_tiles,
-                                              int num_entries) {
+                                              int num_entries, int tail) {
   TileInfo ti;
-  ti.valid = t < num_tiles ? 1 : 0;
-  ti.pad = 0;
-  if (ti.valid) {
+  if (t < num_tiles) {
     const int H = p.num_heads;
-    const int tail = min(H, kTailHeads);
     const int bulk = (H - tail) * num_entries;
     int h, e;
     if (t < bulk) {
@@ -268,17 +292,19 @@ __device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_ti
     ti.Lq = p.cu_q[en.x + 1] - ti.q_start;
     ti.k_start = p.cu_k[en.x];
     ti.Lk = p.cu_k[en.x + 1] - ti.k_start;
+    ti.c_start = p.cu_ctx != nullptr ? p.cu_ctx[en.x] : 0;
+    ti.Lc = p.cu_ctx != nullptr ? p.cu_ctx[en.x + 1] - ti.c_start : 0;
     ti.m0 = en.y * kTileRows;
     ti.h = h;
   } else {
-    ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.m0 = ti.h = 0;
+    ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.c_start = ti.Lc = ti.m0 = ti.h = 0;
   }
   return ti;
 }
 
 __device__ __forceinline__ void tile_blocks(const TileInfo& t, int causal, int (&n)[2]) {
-  n[0] = t.valid ? blocks_for(sub_tile_keys(t.m0, t.Lq, t.Lk, causal)) : 0;
-  n[1] = t.valid ? blocks_for(sub_tile_keys(t.m0 + kSubRows, t.Lq, t.Lk, causal)) : 0;
+  n[0] = sub_tile_blocks(t.m0, t.Lq, t.Lk, t.Lc, causal);
+  n[1] = sub_tile_blocks(t.m0 + kSubRows, t.Lq, t.Lk, t.Lc, causal);
 }
 
 __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
@@ -296,7 +322,9 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
 __global__ void __launch_bounds__(kThreads, 1)
     dense_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_kc,
+                     const __grid_constant__ CUtensorMap tm_vc, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -353,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int causal = p.causal;
   const int num_tiles = p.ws->num_tiles;
   const int num_entries = p.ws->num_entries;
+  const int tail = tail_heads(p.num_heads, num_entries, nclusters);
   auto wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
     return mbar_wait_cluster(bar, parity, abort_flag, err, tlim);
   };
@@ -368,6 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
+      if (p.cu_ctx != nullptr) {
+        prefetch_tensormap(&tm_kc);
+        prefetch_tensormap(&tm_vc);
+      }
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
       int blk = 0;  // KV blocks issued so far (slot = blk % kSlots)
@@ -382,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
           const int t = k == 0 ? cluster : nclusters + atomicAdd(&p.ws->next_tile, 1);
-          ti = tile_info(p, t, num_tiles, num_entries);
+          ti = tile_info(p, t, num_tiles, num_entries, tail);
           // Into both CTAs' slot: the barrier's phase completes once the
           // 32 bytes have landed (st.async counts them on it).
           const uint32_t a = smem_u32(&bars->tiles[ts]);
@@ -390,16 +423,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t fb = mapa_shared(smem_u32(&bars->tile_full[ts]), r);
             mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(sizeof(TileInfo)));
             st_async_v4(mapa_shared(a, r), ti.q_start, ti.Lq, ti.k_start, ti.Lk, fb);
-            st_async_v4(mapa_shared(a + 16, r), ti.m0, ti.h, ti.valid, ti.pad, fb);
+            st_async_v4(mapa_shared(a + 16, r), ti.c_start, ti.Lc, ti.m0, ti.h, fb);
           }
         } else {
           if (!(ok = wait(smem_u32(&bars->tile_full[ts]), tile_par(k),
                           MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
           ti = bars->tiles[ts];
-          if (ti.valid) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
+          if (ti.valid()) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
         }
-        if (!ti.valid) break;
+        if (!ti.valid()) break;
         int nb[2];
         tile_blocks(ti, causal, nb);
         const int nblk = max(nb[0], nb[1]);
@@ -429,10 +462,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_cluster(qbar);
           }
         }
+        const int nctx = blocks_for(ti.Lc);  // the context's blocks come first
         for (int n = 0; n < nblk && ok; ++n, ++blk) {
           const int slot = blk % kSlots;
           const uint32_t par = (static_cast<uint32_t>(blk / kSlots) & 1u) ^ 1u;
-          const int key0 = ti.k_start + n * kBlockKeys;
+          const bool in_ctx = n < nctx;
+          const int key0 = in_ctx ? ti.c_start + n * kBlockKeys
+                                  : ti.k_start + (n - nctx) * kBlockKeys;
+          const CUtensorMap* mk = in_ctx ? &tm_kc : &tm_k;
+          const CUtensorMap* mv = in_ctx ? &tm_vc : &tm_v;
           // K: this CTA's 64 keys, three 64-dim chunks of the 192
           if (!(ok = wait(smem_u32(&bars->empty_k[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
             break;
@@ -442,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kbar = lead(&bars->full_kv[slot]);
 #pragma unroll
           for (int u = 0; u < kKUnits; ++u)
-            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, &tm_k, 64 * u, ti.h,
+            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, mk, 64 * u, ti.h,
                              key0 + static_cast<int>(rank) * kHalfKeys, kbar, pol_kv);
           // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
           if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
@@ -450,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t vbar = kbar;
 #pragma unroll
           for (int u = 0; u < kVUnits; ++u)
-            tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, &tm_v,
+            tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, mv,
                              static_cast<int>(rank) * kHalfDv, ti.h, key0 + 64 * u, vbar, pol_kv);
         }
       }
@@ -528,11 +566,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto fetch = [&](int k, int& valid, int (&n)[2]) -> bool {
         const int ts = tile_slot(k);
         if (!wait_bar(smem_u32(&bars->tile_full[ts]), tile_par(k))) return false;
-        const TileInfo ti = bars->tiles[ts];
+        const TileInfo* t = &bars->tiles[ts];
+        valid = t->valid();
+        n[0] = valid ? sub_tile_blocks(t->m0, t->Lq, t->Lk, t->Lc, causal) : 0;
+        n[1] = valid ? sub_tile_blocks(t->m0 + kSubRows, t->Lq, t->Lk, t->Lc, causal) : 0;
         __syncwarp();
-        if (ti.valid && lane == 0) mbar_arrive(smem_u32(&bars->tile_empty[ts]));
-        valid = ti.valid;
-        tile_blocks(ti, causal, n);
+        if (valid && lane == 0) mbar_arrive(smem_u32(&bars->tile_empty[ts]));
         return true;
       };
 
@@ -629,14 +668,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The block loop needs only the row and key limits; the epilogue reads
       // the tile's coordinates from the slot again (it stays valid until
       // this warp frees it), which keeps them out of registers meanwhile.
-      const TileInfo ti = bars->tiles[ts];
-      if (!ti.valid) break;
-      const int Lk = ti.Lk;
-      const int row0 = ti.m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows;  // this CTA's rows
-      const int r = row0 + wq * 32 + lane;  // row within the sequence
-      const int off = Lk - ti.Lq;
-      const int nb = blocks_for(sub_tile_keys(ti.m0 + sub * kSubRows, ti.Lq, Lk, causal));
-      const int lim = causal ? min(Lk, r + off + 1) : Lk;  // keys [0, lim) visible
+      const TileInfo* slot = &bars->tiles[ts];
+      if (!slot->valid()) break;
+      const int Lk = slot->Lk;
+      const int Lc = slot->Lc;
+      const int nc = blocks_for(Lc);  // context blocks (every context key is visible)
+      // first row of this CTA's part of the sub-tile, and the last own key
+      // that row sees (bottom-right causal: row i sees keys j <= i + Lk - Lq)
+      const int row0 = slot->m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows;
+      const int diag = row0 + Lk - slot->Lq;
+      const int nb = sub_tile_blocks(slot->m0 + sub * kSubRows, slot->Lq, Lk, Lc, causal);
+      const int ldiag = diag + wq * 32 + lane;  // this thread's row's last key
+      const int lim = causal ? min(Lk, ldiag + 1) : Lk;  // own keys [0, lim) visible
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
       float l_run = 0.f;        // running sum of the fp32 weights exp2(scaled s - m_run)
 
@@ -651,13 +694,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(sraw[j]);
-        const int kbase = n * kBlockKeys;
-        const bool full_blk = (kbase + kBlockKeys <= Lk) &&
-                              (!causal || kbase + kBlockKeys - 1 <= row0 + off);
+        // Blocks [0, nc) hold context keys 128 n + j, visible below Lc; the
+        // sequence's own keys follow, visible below the row's limit.  A block
+        // that every row of the CTA sees whole needs no mask.
+        const bool in_ctx = n < nc;
+        const int kbase = (in_ctx ? n : n - nc) * kBlockKeys;
+        const bool full_blk =
+            in_ctx ? kbase + kBlockKeys <= Lc
+                   : (kbase + kBlockKeys <= Lk) && (!causal || kbase + kBlockKeys - 1 <= diag);
         if (!full_blk) {
+          const int klim = in_ctx ? Lc : lim;
 #pragma unroll
           for (int j = 0; j < 128; ++j)
-            if (kbase + j >= lim) x[j] = -INFINITY;
+            if (kbase + j >= klim) x[j] = -INFINITY;
         }
         float m8[8];
 #pragma unroll
@@ -711,6 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e_lq = bars->tiles[ts].Lq;
       const int e_q0 = bars->tiles[ts].q_start;
       const int e_h = bars->tiles[ts].h;
+      const int r = bars->tiles[ts].m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows +
+                    wq * 32 + lane;  // this thread's row within the sequence
       // Done with the tile's ring slot.  Freed here rather than at the start
       // of the tile so that the cluster-scope release does not wait for the
       // previous epilogue's stores.
@@ -718,10 +769,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
 
       // ------------------------------------------------------- epilogue
+      // Denominator Z = l 2^m (+ 2^s for the head's sink s, in the same log2
+      // units); O = O_acc 2^m / Z, LSE = log2(Z) ln 2.  Without a sink this
+      // is O_acc / l and m + log2 l.  A row that saw no key keeps m_run =
+      // -inf (its weights are only the tiny clamped values of the polynomial
+      // path): output 0, LSE -inf, or the sink's logit.
       const bool row_ok = r < e_lq;
       const size_t row_index = static_cast<size_t>(e_q0 + r) * p.num_heads + e_h;
-      uint4* orow = reinterpret_cast<uint4*>(p.out + row_index * kDv);
-      float lse_val = -INFINITY;
+      const bool fp8 = p.out_scale != nullptr;
+      const float sink2 = p.sinks != nullptr ? p.sinks[e_h] * 1.4426950408889634f : -INFINITY;
+      float lse2 = sink2;  // log2 of the row's denominator
       if (nb > 0) {
         ok = __all_sync(0xffffffffu, wait(smem_u32(&bars->o_full[sub]),
                                           static_cast<uint32_t>(o_cnt) & 1u,
@@ -734,28 +791,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(obar_lead);  // O may be overwritten now
         ++o_cnt;
-        // A row that saw no key keeps m_run = -inf (its weights are only the
-        // tiny clamped values of the polynomial path): output 0, LSE -inf.
-        const bool seen = m_run != -INFINITY;
-        const float inv = seen ? 1.0f / l_run : 0.0f;
-        if (row_ok) {
+        float scale_o = 0.0f;  // multiplier of O's accumulator
+        if (m_run != -INFINITY) {
+          if (p.sinks == nullptr) {
+            scale_o = 1.0f / l_run;
+            lse2 = m_run + lg2_approx(l_run);
+          } else {
+            const float mz = fmaxf(m_run, sink2);
+            const float z = l_run * ex2_approx(m_run - mz) + ex2_approx(sink2 - mz);
+            scale_o = ex2_approx(m_run - mz) / z;
+            lse2 = mz + lg2_approx(z);
+          }
+        }
+        if (row_ok && !fp8) {
+          uint4* orow =
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_index * kDv);
 #pragma unroll
           for (int v4 = 0; v4 < 16; ++v4) {
             uint32_t pk[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
-                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv);
+              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * scale_o,
+                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * scale_o);
             orow[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-        }
-        if (seen) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
-      } else if (row_ok) {
+        } else if (row_ok) {
+          // e4m3 of O / out_scale: round to nearest even, saturated at 448
+          const float qs = scale_o / *p.out_scale;
+          uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row_index * kDv);
 #pragma unroll
-        for (int v4 = 0; v4 < 16; ++v4) orow[v4] = make_uint4(0u, 0u, 0u, 0u);
+          for (int v16 = 0; v16 < 8; ++v16) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              pk[j] = pack_e4m3x4(__uint_as_float(o[16 * v16 + 4 * j]) * qs,
+                                  __uint_as_float(o[16 * v16 + 4 * j + 1]) * qs,
+                                  __uint_as_float(o[16 * v16 + 4 * j + 2]) * qs,
+                                  __uint_as_float(o[16 * v16 + 4 * j + 3]) * qs);
+            orow[v16] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      } else if (row_ok) {
+        // no visible key: zeros (bf16 rows of 256 bytes, e4m3 rows of 128)
+        uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
+                                               row_index * kDv * (fp8 ? 1 : 2));
+        const int n16 = fp8 ? 8 : 16;
+        for (int v = 0; v < n16; ++v) orow[v] = make_uint4(0u, 0u, 0u, 0u);
       }
       if (row_ok && p.lse != nullptr)
-        p.lse[static_cast<size_t>(e_h) * p.total_q + e_q0 + r] = lse_val;
+        p.lse[static_cast<size_t>(e_h) * p.total_q + e_q0 + r] = lse2 * 0.69314718055994530942f;
     }
   }
 

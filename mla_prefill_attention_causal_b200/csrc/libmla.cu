@@ -305,6 +305,163 @@ size_t mla_prefill_workspace_size(int batch, int total_q) {
   return mla::dense::kWsHeaderBytes + entries * sizeof(int2);
 }
 
+}  // extern "C"
+
+namespace {
+
+// One dense prefill call: the arguments of every dense entry point.  The
+// context (k_ctx, v_ctx, cu_ctx), the sinks and the output scale are
+// optional (null).
+struct DenseCall {
+  const void* q;
+  int64_t q_rs, q_hs;
+  const void* k;
+  int64_t k_rs, k_hs;
+  const void* v;
+  int64_t v_rs, v_hs;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const void* k_ctx = nullptr;
+  const void* v_ctx = nullptr;
+  const int32_t* cu_ctx = nullptr;
+  int max_ctx = 0, total_ctx = 0;
+  const float* sinks = nullptr;
+  const float* out_scale = nullptr;
+  int max_q, max_k;
+  float scale;
+  int causal;
+  void* out;
+  float* lse;
+  mla_stream_t stream;
+  int batch, num_heads, total_q, total_k;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+int dense_call(const DenseCall& c) {
+  using namespace mla::dense;
+  if (c.q == nullptr || c.k == nullptr || c.v == nullptr || c.cu_q == nullptr ||
+      c.cu_k == nullptr || c.out == nullptr || c.workspace == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(c.q, 16) || !aligned(c.k, 16) || !aligned(c.v, 16) || !aligned(c.out, 16) ||
+      !aligned(c.workspace, 16) || !aligned(c.cu_q, 4) || !aligned(c.cu_k, 4) ||
+      (c.lse && !aligned(c.lse, 4)) || (c.sinks && !aligned(c.sinks, 4)) ||
+      (c.out_scale && !aligned(c.out_scale, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (c.batch < 1 || c.num_heads < 1 || c.num_heads > 65535 || c.total_q < 0 || c.total_k < 0 ||
+      c.max_q < 0 || c.max_k < 0 || (c.causal != 0 && c.causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(c.scale) || !(c.scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  if (!good_stride(c.q_rs) || !good_stride(c.q_hs) || !good_stride(c.k_rs) ||
+      !good_stride(c.k_hs) || !good_stride(c.v_rs) || !good_stride(c.v_hs))
+    return MLA_ERR_INVALID_ARG;
+  const bool ctx = c.cu_ctx != nullptr || c.k_ctx != nullptr || c.v_ctx != nullptr;
+  if (ctx && (c.cu_ctx == nullptr || c.k_ctx == nullptr || c.v_ctx == nullptr ||
+              !aligned(c.k_ctx, 16) || !aligned(c.v_ctx, 16) || !aligned(c.cu_ctx, 4) ||
+              c.total_ctx < 0 || c.max_ctx < 0))
+    return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_prefill_workspace_size(c.batch, c.total_q);
+  if (c.workspace_bytes < need) return MLA_ERR_INVALID_ARG;
+  // the kernels count tiles (work-list entries x heads, plus one grab per
+  // cluster past the end) in int
+  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * c.num_heads >
+      INT32_MAX - 65536)
+    return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  int st = prepare_device(&dev);
+  if (st != MLA_OK) return st;
+  if (c.total_q == 0) return MLA_OK;  // nothing to compute
+
+  CUtensorMap tq, tk, tv, tkc, tvc;
+  const uint64_t kv_rows = c.total_k > 0 ? static_cast<uint64_t>(c.total_k) : 1;
+  const uint64_t H = static_cast<uint64_t>(c.num_heads);
+  if ((st = encode_heads(&tq, c.q, kDqk, H, static_cast<uint64_t>(c.total_q), c.q_hs, c.q_rs,
+                         kCtaRows)) != MLA_OK ||
+      (st = encode_heads(&tk, c.k, kDqk, H, kv_rows, c.k_hs, c.k_rs, kHalfKeys)) != MLA_OK ||
+      (st = encode_heads(&tv, c.v, kDv, H, kv_rows, c.v_hs, c.v_rs, 64)) != MLA_OK)
+    return st;
+  if (ctx) {
+    // the context is packed: [total_ctx, H, 192] and [total_ctx, H, 128]
+    const uint64_t c_rows = c.total_ctx > 0 ? static_cast<uint64_t>(c.total_ctx) : 1;
+    const int64_t hs = c.num_heads;
+    if ((st = encode_heads(&tkc, c.k_ctx, kDqk, H, c_rows, kDqk, hs * kDqk, kHalfKeys)) !=
+            MLA_OK ||
+        (st = encode_heads(&tvc, c.v_ctx, kDv, H, c_rows, kDv, hs * kDv, 64)) != MLA_OK)
+      return st;
+  } else {
+    tkc = tk;  // not read: every sequence has an empty context
+    tvc = tv;
+  }
+
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(c.stream);
+  WsHeader* ws = static_cast<WsHeader*>(c.workspace);
+  int2* entries = reinterpret_cast<int2*>(static_cast<char*>(c.workspace) + kWsHeaderBytes);
+  const int capacity = static_cast<int>((need - kWsHeaderBytes) / sizeof(int2));
+  dense_plan_kernel<<<1, kPlanThreads, 0, s>>>(c.cu_q, c.cu_k, c.cu_ctx, c.batch, c.causal, ws,
+                                               entries, capacity, c.num_heads);
+  if ((st = launch_status()) != MLA_OK) return st;
+
+  Params p;
+  p.cu_q = c.cu_q;
+  p.cu_k = c.cu_k;
+  p.cu_ctx = c.cu_ctx;
+  p.out = c.out;
+  p.lse = c.lse;
+  p.sinks = c.sinks;
+  p.out_scale = c.out_scale;
+  p.ws = ws;
+  p.entries = entries;
+  p.num_heads = c.num_heads;
+  p.total_q = c.total_q;
+  p.causal = c.causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634074);
+  p.timeout_ns = wait_timeout_ns();
+  // Persistent: as many 2-CTA clusters as can be resident at once, but never
+  // more than tiles could exist.
+  const long long max_tiles = static_cast<long long>(capacity) * c.num_heads;
+  const long long resident = g_dev[dev].dense_clusters.load(std::memory_order_relaxed);
+  const long long clusters = max_tiles < resident ? max_tiles : resident;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dense_fwd_kernel, tq, tk, tv, tkc, tvc, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// The call over packed q [T, H, 192], k [Tk, H, 192], v [Tk, H, 128].
+DenseCall packed_call(const void* q, const void* k, const void* v, int num_heads) {
+  using mla::dense::kDqk;
+  using mla::dense::kDv;
+  DenseCall c;
+  const int64_t H = num_heads;
+  c.q = q;
+  c.q_rs = H * kDqk;
+  c.q_hs = kDqk;
+  c.k = k;
+  c.k_rs = H * kDqk;
+  c.k_hs = kDqk;
+  c.v = v;
+  c.v_rs = H * kDv;
+  c.v_hs = kDv;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
 int mla_prefill_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
                     const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
                     float softmax_scale, int causal, void* out, float* lse, mla_stream_t stream,
@@ -326,85 +483,92 @@ int mla_prefill_fwd_strided(const void* q, int64_t q_row_stride, int64_t q_head_
                             int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
                             void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
                             int total_q, int total_k, void* workspace, size_t workspace_bytes) {
-  using namespace mla::dense;
-  if (q == nullptr || k == nullptr || v == nullptr || cu_seqlens_q == nullptr ||
-      cu_seqlens_k == nullptr || out == nullptr || workspace == nullptr)
-    return MLA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      !aligned(workspace, 16) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
-      (lse && !aligned(lse, 4)))
-    return MLA_ERR_INVALID_ARG;
-  if (batch < 1 || num_heads < 1 || num_heads > 65535 || total_q < 0 || total_k < 0 ||
-      max_seqlen_q < 0 || max_seqlen_k < 0 || (causal != 0 && causal != 1))
-    return MLA_ERR_INVALID_ARG;
-  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
-  if (!good_stride(q_row_stride) || !good_stride(q_head_stride) || !good_stride(k_row_stride) ||
-      !good_stride(k_head_stride) || !good_stride(v_row_stride) || !good_stride(v_head_stride))
-    return MLA_ERR_INVALID_ARG;
-  const size_t need = mla_prefill_workspace_size(batch, total_q);
-  if (workspace_bytes < need) return MLA_ERR_INVALID_ARG;
-  // the kernels count tiles (work-list entries x heads, plus one grab per
-  // cluster past the end) in int
-  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * num_heads >
-      INT32_MAX - 65536)
-    return MLA_ERR_INVALID_ARG;
-  int dev = 0;
-  int st = prepare_device(&dev);
-  if (st != MLA_OK) return st;
-  if (total_q == 0) return MLA_OK;  // nothing to compute
+  DenseCall c;
+  c.q = q;
+  c.q_rs = q_row_stride;
+  c.q_hs = q_head_stride;
+  c.k = k;
+  c.k_rs = k_row_stride;
+  c.k_hs = k_head_stride;
+  c.v = v;
+  c.v_rs = v_row_stride;
+  c.v_hs = v_head_stride;
+  c.cu_q = cu_seqlens_q;
+  c.cu_k = cu_seqlens_k;
+  c.max_q = max_seqlen_q;
+  c.max_k = max_seqlen_k;
+  c.scale = softmax_scale;
+  c.causal = causal;
+  c.out = out;
+  c.lse = lse;
+  c.stream = stream;
+  c.batch = batch;
+  c.num_heads = num_heads;
+  c.total_q = total_q;
+  c.total_k = total_k;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  return dense_call(c);
+}
 
-  CUtensorMap tq, tk, tv;
-  const uint64_t kv_rows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
-  const uint64_t H = static_cast<uint64_t>(num_heads);
-  if ((st = encode_heads(&tq, q, kDqk, H, static_cast<uint64_t>(total_q), q_head_stride,
-                         q_row_stride, kCtaRows)) != MLA_OK ||
-      (st = encode_heads(&tk, k, kDqk, H, kv_rows, k_head_stride, k_row_stride, kHalfKeys)) !=
-          MLA_OK ||
-      (st = encode_heads(&tv, v, kDv, H, kv_rows, v_head_stride, v_row_stride, 64)) != MLA_OK)
-    return st;
+int mla_prefill_fwd_context(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            const void* k_ctx, const void* v_ctx, const int32_t* cu_seqlens_ctx,
+                            int max_seqlen_q, int max_seqlen_k, int max_seqlen_ctx,
+                            float softmax_scale, int causal, void* out, float* lse,
+                            mla_stream_t stream, int batch, int num_heads, int total_q,
+                            int total_k, int total_ctx, void* workspace, size_t workspace_bytes) {
+  if (k_ctx == nullptr || v_ctx == nullptr || cu_seqlens_ctx == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  DenseCall c = packed_call(q, k, v, num_heads);
+  c.cu_q = cu_seqlens_q;
+  c.cu_k = cu_seqlens_k;
+  c.k_ctx = k_ctx;
+  c.v_ctx = v_ctx;
+  c.cu_ctx = cu_seqlens_ctx;
+  c.max_ctx = max_seqlen_ctx;
+  c.total_ctx = total_ctx;
+  c.max_q = max_seqlen_q;
+  c.max_k = max_seqlen_k;
+  c.scale = softmax_scale;
+  c.causal = causal;
+  c.out = out;
+  c.lse = lse;
+  c.stream = stream;
+  c.batch = batch;
+  c.num_heads = num_heads;
+  c.total_q = total_q;
+  c.total_k = total_k;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  return dense_call(c);
+}
 
-  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  WsHeader* ws = static_cast<WsHeader*>(workspace);
-  int2* entries = reinterpret_cast<int2*>(static_cast<char*>(workspace) + kWsHeaderBytes);
-  const int capacity = static_cast<int>((need - kWsHeaderBytes) / sizeof(int2));
-  dense_plan_kernel<<<1, kPlanThreads, 0, s>>>(cu_seqlens_q, cu_seqlens_k, batch, causal, ws,
-                                               entries, capacity, num_heads);
-  if ((st = launch_status()) != MLA_OK) return st;
-
-  Params p;
-  p.cu_q = cu_seqlens_q;
-  p.cu_k = cu_seqlens_k;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.ws = ws;
-  p.entries = entries;
-  p.num_heads = num_heads;
-  p.total_q = total_q;
-  p.causal = causal;
-  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
-  p.timeout_ns = wait_timeout_ns();
-  // Persistent: as many 2-CTA clusters as can be resident at once, but never
-  // more than tiles could exist.
-  const long long max_tiles = static_cast<long long>(capacity) * num_heads;
-  const long long resident = g_dev[dev].dense_clusters.load(std::memory_order_relaxed);
-  const long long clusters = max_tiles < resident ? max_tiles : resident;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, dense_fwd_kernel, tq, tk, tv, p) != cudaSuccess) {
-    cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
-  return launch_status();
+int mla_prefill_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                       const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+                       float softmax_scale, int causal, const float* sinks,
+                       const float* output_scale, void* out, float* lse, mla_stream_t stream,
+                       int batch, int num_heads, int total_q, int total_k, void* workspace,
+                       size_t workspace_bytes) {
+  DenseCall c = packed_call(q, k, v, num_heads);
+  c.cu_q = cu_seqlens_q;
+  c.cu_k = cu_seqlens_k;
+  c.sinks = sinks;
+  c.out_scale = output_scale;
+  c.max_q = max_seqlen_q;
+  c.max_k = max_seqlen_k;
+  c.scale = softmax_scale;
+  c.causal = causal;
+  c.out = out;
+  c.lse = lse;
+  c.stream = stream;
+  c.batch = batch;
+  c.num_heads = num_heads;
+  c.total_q = total_q;
+  c.total_k = total_k;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  return dense_call(c);
 }
 
 int mla_prefill_fwd_noalloc(const void* q, const void* k, const void* v,

@@ -162,3 +162,38 @@ def test_python_binding_checks_arguments_before_any_launch():
                                    torch.zeros((4, 16), dtype=torch.int32))
     with pytest.raises(ValueError, match="CUDA device"):
         mla.mla_attn_merge(v, torch.zeros((2, 4)), v, torch.zeros((2, 4)))
+
+
+def _call_context(**over):
+    a = dict(q=16, k=16, v=16, cq=16, ck=16, kc=32, vc=32, cc=16, mq=4, mk=4, mc=4, scale=0.1,
+             causal=1, out=16, lse=None, batch=1, H=1, tq=4, tk=4, tc=4, ws=64, wsb=4096)
+    a.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return mla.load().mla_prefill_fwd_context(
+        P(a["q"]), P(a["k"]), P(a["v"]), P(a["cq"]), P(a["ck"]), P(a["kc"]), P(a["vc"]),
+        P(a["cc"]), a["mq"], a["mk"], a["mc"], a["scale"], a["causal"], P(a["out"]), P(a["lse"]),
+        None, a["batch"], a["H"], a["tq"], a["tk"], a["tc"], P(a["ws"]), a["wsb"])
+
+
+@pytest.mark.parametrize("over", [dict(kc=None), dict(vc=None), dict(cc=None), dict(kc=40),
+                                  dict(vc=24), dict(cc=2), dict(tc=-1), dict(mc=-1), dict(q=None),
+                                  dict(wsb=100), dict(causal=3)])
+def test_context_call_rejects_bad_arguments(over):
+    assert _call_context(**over) == _lib.MLA_ERR_INVALID_ARG
+
+
+def _call_ex(**over):
+    a = dict(q=16, k=16, v=16, cq=16, ck=16, mq=4, mk=4, scale=0.1, causal=1, sinks=None,
+             osc=None, out=16, lse=None, batch=1, H=1, tq=4, tk=4, ws=64, wsb=4096)
+    a.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return mla.load().mla_prefill_fwd_ex(
+        P(a["q"]), P(a["k"]), P(a["v"]), P(a["cq"]), P(a["ck"]), a["mq"], a["mk"], a["scale"],
+        a["causal"], P(a["sinks"]), P(a["osc"]), P(a["out"]), P(a["lse"]), None, a["batch"],
+        a["H"], a["tq"], a["tk"], P(a["ws"]), a["wsb"])
+
+
+@pytest.mark.parametrize("over", [dict(sinks=2), dict(osc=6), dict(out=None), dict(out=8),
+                                  dict(scale=0.0), dict(H=0)])
+def test_ex_call_rejects_bad_arguments(over):
+    assert _call_ex(**over) == _lib.MLA_ERR_INVALID_ARG

@@ -225,3 +225,146 @@ def chunked_concat(d):
     v_cat = np.concatenate([np.concatenate([d["v_prefix"][b * P:(b + 1) * P],
                                             d["v_self"][b * C:(b + 1) * C]]) for b in range(B)])
     return k_cat, v_cat, syn.cu_seqlens([P + C] * B)
+
+
+# ----------------------------------------------------------------- context pass
+def _context_call(q, k, v, cu_q, cu_k, kc, vc, cu_c, scale, causal):
+    import mla_prefill_attention_causal_b200 as mla
+    lq, lk, lc = np.diff(cu_q), np.diff(cu_k), np.diff(cu_c)
+    out, lse = mla.mla_prefill_fwd_context(
+        dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_i32(cu_q), dev_i32(cu_k), dev_bf16(kc),
+        dev_bf16(vc), dev_i32(cu_c), int(lq.max()), int(lk.max()), int(lc.max()), scale,
+        causal=causal)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_context_pass_matches_merge_of_context_and_own_keys(causal):
+    """The one-pass chunked prefill equals the oracle's merge of an unmasked
+    pass over the context and a pass over the sequence's own keys, on a
+    ragged batch: contexts of 700, 0, 129, 1, 128 and 127 keys, a sequence
+    with more queries than keys and one without keys of its own."""
+    lens_q = [300, 129, 1, 513, 200, 64]
+    lens_k = [300, 129, 1, 513, 150, 0] if causal else [256, 40, 7, 600, 150, 0]
+    lens_c = [700, 0, 129, 1, 128, 127]
+    H = 4
+    case = syn.dense_case(lens_q, lens_k, H, seed=81, causal=causal)
+    ctx = syn.dense_case(lens_c, lens_c, H, seed=82)
+    out, lse = _context_call(case["q"], case["k"], case["v"], case["cu_q"], case["cu_k"],
+                             ctx["k"], ctx["v"], ctx["cu_k"], case["scale"], causal)
+    o_c, l_c = oracle.dense_prefill(case["q"], ctx["k"], ctx["v"], case["cu_q"], ctx["cu_k"],
+                                    case["scale"], False)
+    o_s, l_s = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"], case["cu_k"],
+                                    case["scale"], causal)
+    ref_o, ref_l = oracle.attn_merge(o_c, l_c, o_s, l_s)
+    assert_out_close(to_f64(out), ref_o, "context out")
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), ref_l, "context lse")
+
+
+def test_context_pass_without_context_is_the_plain_call():
+    """Empty contexts: bit for bit the result of mla_prefill_fwd."""
+    lens = [700, 129, 300]
+    case = syn.dense_case(lens, lens, 4, seed=83)
+    kc = np.zeros((1, 4, 192), dtype=case["k"].dtype)  # a real (unread) buffer
+    vc = np.zeros((1, 4, 128), dtype=case["v"].dtype)
+    out, lse = _context_call(case["q"], case["k"], case["v"], case["cu_q"], case["cu_k"], kc, vc,
+                             syn.cu_seqlens([0, 0, 0]), case["scale"], True)
+    o_p, l_p = run_dense(case)
+    assert torch.equal(out, o_p) and torch.equal(lse, l_p)
+
+
+def test_context_pass_chunked_workload_full():
+    """The chunked workload (4 x 2048 new tokens over 16384-token contexts,
+    128 heads) in one pass: every row of 33 heads against one bottom-right
+    causal oracle call over each sequence's [context, chunk] keys."""
+    d = syn.chunked_config()
+    out, lse = _context_call(d["q"], d["k_self"], d["v_self"], d["cu_q"], d["cu_q"],
+                             d["k_prefix"], d["v_prefix"], d["cu_prefix"], d["scale"], True)
+    k_cat, v_cat, cu_cat = chunked_concat(d)
+    check_dense_full("chunked in one pass (mla_prefill_fwd_context, 33 heads)", d["q"], k_cat,
+                     v_cat, d["cu_q"], cu_cat, d["scale"], True, out, lse,
+                     heads=CHUNKED_HEADS, heads_per_job=1)
+
+
+# ------------------------------------------------------- sinks and e4m3 output
+def _run_ex(case, sinks=None, output_scale=None):
+    import mla_prefill_attention_causal_b200 as mla
+    s = None if sinks is None else torch.tensor(sinks, dtype=torch.float32, device="cuda")
+    o_s = None if output_scale is None else torch.tensor([output_scale], dtype=torch.float32,
+                                                         device="cuda")
+    out, lse = mla.mla_prefill_fwd_ex(dev_bf16(case["q"]), dev_bf16(case["k"]), dev_bf16(case["v"]),
+                                      dev_i32(case["cu_q"]), dev_i32(case["cu_k"]), case["max_q"],
+                                      case["max_k"], case["scale"], causal=case["causal"], sinks=s,
+                                      output_scale=o_s)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def test_ex_without_options_is_the_plain_call():
+    case = syn.dense_case([700, 129, 300], [700, 129, 300], 4, seed=95)
+    o, l = _run_ex(case)
+    o_p, l_p = run_dense(case)
+    assert torch.equal(o, o_p) and torch.equal(l, l_p)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_sinks_match_oracle(causal):
+    """One sink logit per head (two of them far above every score) on a
+    ragged batch that has rows without any key (O = 0, LSE = the sink)."""
+    lens_q = [300, 129, 1, 200]
+    lens_k = [300, 129, 1, 150] if causal else [256, 40, 7, 0]
+    case = syn.dense_case(lens_q, lens_k, 4, seed=96, causal=causal)
+    sinks = np.array([0.5, -1.5, 12.0, 3.0], dtype=np.float32)
+    out, lse = _run_ex(case, sinks=sinks)
+    ref_o, ref_l = oracle.dense_prefill_sinks(case["q"], case["k"], case["v"], case["cu_q"],
+                                              case["cu_k"], case["scale"], causal,
+                                              sinks.astype(np.float64))
+    assert_out_close(to_f64(out), ref_o, "sink out")
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), ref_l, "sink lse")
+
+
+def _e4m3_step(y):
+    """Spacing of the e4m3 grid around |y| (2^-9 below the normal range)."""
+    a = np.minimum(np.abs(y), 448.0)
+    return np.exp2(np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3.0)
+
+
+@pytest.mark.parametrize("scale", [0.01, 0.25, 1e-4])
+def test_fp8_output_is_the_e4m3_of_the_same_output(scale):
+    """e4m3 output of O / scale.  The kernel rounds the same fp32 O that its
+    bf16 output rounds, so each code lies within one e4m3 step of that bf16
+    value / scale (the bf16 rounding is far finer than the e4m3 grid), and
+    within the bf16 tolerance plus one step of the oracle.  The LSE is the
+    plain call's, bit for bit.  Scale 1e-4 saturates most outputs at 448."""
+    case = syn.dense_case([513, 130, 1], [513, 130, 1], 4, seed=97)
+    out, lse = _run_ex(case, output_scale=scale)
+    assert out.dtype == torch.float8_e4m3fn
+    got = oracle.e4m3_decode(out.view(torch.uint8).cpu().numpy())
+    o_p, l_p = run_dense(case)
+    assert torch.equal(lse, l_p)
+    y_b = np.clip(to_f64(o_p) / np.float64(scale), -448.0, 448.0)
+    assert np.all(np.abs(got - y_b) <= _e4m3_step(y_b) * 1.0001)
+    ref_o, _ = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"], case["cu_k"],
+                                    case["scale"], True)
+    y = ref_o / np.float64(scale)
+    err = np.abs(got - np.clip(y, -448.0, 448.0))
+    assert np.all(err <= 2e-2 / scale + _e4m3_step(y) * 1.0001)
+    # saturated where the exact value is clearly out of range
+    sat = np.abs(y) > 448.0 * 1.01
+    assert np.all(np.abs(got[sat]) == 448.0)
+    # the bulk of the codes are the oracle's own rounding
+    assert np.mean(oracle.e4m3_quantize(ref_o, scale) ==
+                   out.view(torch.uint8).cpu().numpy()) > 0.9
+
+
+def test_sinks_with_fp8_output():
+    """Both options at once: the e4m3 codes of the sink-weighted output."""
+    case = syn.dense_case([257, 64], [257, 64], 2, seed=98)
+    sinks = np.array([1.0, -0.5], dtype=np.float32)
+    out, lse = _run_ex(case, sinks=sinks, output_scale=0.02)
+    o_b, l_b = _run_ex(case, sinks=sinks)
+    assert torch.equal(lse, l_b)
+    got = oracle.e4m3_decode(out.view(torch.uint8).cpu().numpy())
+    y_b = np.clip(to_f64(o_b) / 0.02, -448.0, 448.0)
+    assert np.all(np.abs(got - y_b) <= _e4m3_step(y_b) * 1.0001)

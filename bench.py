@@ -8,14 +8,16 @@ causal, fp32 LSE.  Throughput counts causal-adjusted algorithmic FLOPs:
 2 * (192 + 128) * heads * (visible query-key pairs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--workload dense|long32k|chunked|chunked-context|sparse|sparse-padded]
+                  [--workload dense|long32k|chunked|chunked-context|splitkv|sparse|
+                              sparse-padded]
 
 ``--workload long32k`` times one 32768-token causal sequence (128 heads);
 ``--workload chunked`` times the chunked prefill with context (a non-causal
 prefix pass, a causal self pass and ``mla_attn_merge``; the merge is also
 event-timed on its own against the HBM roofline), ``--workload
 chunked-context`` the same in one ``mla_prefill_fwd_context`` call;
-``--workload sparse``
+``--workload splitkv`` a few-tile shape (16 heads, 129 queries over 8192
+keys) through ``mla_prefill_fwd_splitkv``; ``--workload sparse``
 times the absorbed top-k path instead: one ``mla_sparse_prefill_fwd`` call
 over 4096 tokens x 128 heads (q dim 576), a 32768-row latent cache and
 top-k 2048 (``sparse-padded``: the same with the tokens at the start of the
@@ -505,6 +507,105 @@ class ChunkedContextWorkload(ChunkedWorkload):
         return cfg
 
 
+class SplitKvWorkload(DenseWorkload):
+    """A few-tile shape: 16 heads (a tensor-parallel share of 128), one
+    sequence of 129 queries (the vLLM warmup probe) over 8192 keys,
+    bottom-right causal, through ``mla_prefill_fwd_splitkv`` with the
+    library's choice of splits; the same call without splits is timed
+    beside it (``config.unsplit_ms``)."""
+
+    metric = ("MLA prefill attn TFLOPS (causal-adj), split-KV on a few-tile shape, "
+              "% of B200 dense BF16 peak, 1 GPU")
+    profile = "dense_fwd_splitkv.md"
+
+    def __init__(self, dev, seed, heads):
+        import torch
+        import mla_synth as syn
+        import oracle
+        import mla_prefill_attention_causal_b200 as mla
+        self.long = False
+        self.name = "splitkv"
+        H = 16 if heads == 128 else heads
+        self.case = case = syn.dense_case([129], [8192], H, seed)
+        self.H = H
+        self.flops = oracle.dense_flops(case["lens_q"], case["lens_k"], H, True)
+        to_t = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+        self.hin = [to_t(case["q"]).pin_memory(), to_t(case["k"]).pin_memory(),
+                    to_t(case["v"]).pin_memory(), torch.from_numpy(case["cu_q"]).pin_memory(),
+                    torch.from_numpy(case["cu_k"]).pin_memory()]
+        self.q, self.k, self.v, self.cu, self.cuk = [x.to(dev) for x in self.hin]
+        T = self.T = self.q.shape[0]
+        self.out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        self.hout = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory(),
+                     torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.splits = mla.num_splits_for(1, T, H, case["max_q"], case["max_k"])
+        self.ws = torch.empty(mla.splitkv_workspace_size(1, T, H, self.splits), dtype=torch.uint8,
+                              device=dev)
+        self.launches = 3 if self.splits > 1 else 2
+        self.unsplit_ms = None
+
+    def _call(self, splits, ws=None):
+        import mla_prefill_attention_causal_b200 as mla
+        c = self.case
+        mla.mla_prefill_fwd_splitkv(self.q, self.k, self.v, self.cu, self.cuk, c["max_q"],
+                                    c["max_k"], c["scale"], causal=True, num_splits=splits,
+                                    out=self.out, lse=self.lse, workspace=ws)
+
+    def step(self):
+        self._call(self.splits, self.ws)
+
+    def e2e_step(self):
+        for d, h in zip((self.q, self.k, self.v, self.cu, self.cuk), self.hin):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.hout[0].copy_(self.out, non_blocking=True)
+        self.hout[1].copy_(self.lse, non_blocking=True)
+
+    def time_unsplit(self, steps):
+        import torch
+        for _ in range(3):
+            self._call(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            self._call(1)
+        e1.record()
+        torch.cuda.synchronize()
+        self.unsplit_ms = e0.elapsed_time(e1) / steps
+
+    def config(self):
+        c = self.case
+        return {"workload": ("split-KV few-tile shape: 1 sequence of 129 queries over 8192 keys, "
+                             "bottom-right causal, %d heads, qk 192 / v 128, bf16 N(0,1), scale "
+                             "1/sqrt(192)" % self.H),
+                "heads": self.H, "num_splits": self.splits, "flops_per_step": self.flops,
+                "unsplit_ms": self.unsplit_ms,
+                "l2": "inputs %.1f MB < L2: repeated calls read K/V from L2 (a launch-bound "
+                      "shape)" % ((self.q.numel() + self.k.numel() + self.v.numel()) * 2 / 1e6)}
+
+    data = "synthetic (seeded N(0,1) bf16)"
+
+    def oracle_sample(self):
+        import oracle
+        c = self.case
+        t0 = time.perf_counter()
+        oracle.dense_prefill(c["q"], c["k"], c["v"], c["cu_q"], c["cu_k"], c["scale"], True)
+        dt = time.perf_counter() - t0
+        return self.flops, dt, f"the whole call ({self.flops:.3e} FLOPs in {dt:.1f} s)"
+
+    def reference_step(self, i):
+        import oracle
+        c = self.case
+        h = i % self.H
+        t0 = time.perf_counter()
+        oracle.dense_prefill(c["q"][:, h:h + 1], c["k"][:, h:h + 1], c["v"][:, h:h + 1],
+                             c["cu_q"], c["cu_k"], c["scale"], True)
+        return oracle.dense_flops(c["lens_q"], c["lens_k"], 1, True), time.perf_counter() - t0
+
+    reference_sample = "step i = head (i mod 16) of the whole call"
+
+
 def rank_seed(base: int, rank: int, world: int) -> int:
     """Seed of a rank's batch: the workload's own seed on one GPU, and a
     distinct batch per rank under weak scaling."""
@@ -535,6 +636,8 @@ def make(args, dev, rank, world):
         return ChunkedWorkload(dev, rank_seed(4, rank, world), args.heads)
     if args.workload == "chunked-context":
         return ChunkedContextWorkload(dev, rank_seed(4, rank, world), args.heads)
+    if args.workload == "splitkv":
+        return SplitKvWorkload(dev, rank_seed(6, rank, world), args.heads)
     return SparseWorkload(dev, rank_seed(5, rank, world), args.heads,
                           padded=args.workload == "sparse-padded")
 
@@ -543,7 +646,12 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
     # The reference arm runs the oracle on the host only: build the host-side case.
-    if args.workload in ("dense", "long32k"):
+    if args.workload == "splitkv":
+        import mla_synth as syn
+        w = SplitKvWorkload.__new__(SplitKvWorkload)
+        w.H = 16
+        w.case = syn.dense_case([129], [8192], w.H, 6)
+    elif args.workload in ("dense", "long32k"):
         w = DenseWorkload.__new__(DenseWorkload)
         w.long = args.workload == "long32k"
         w.case = make_workload(3 if w.long else 2, long=w.long)
@@ -618,6 +726,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
+    if hasattr(w, "time_unsplit"):
+        w.time_unsplit(args.steps)  # outside the timed region, for comparison
     merge_ms = None
     if getattr(w, "merge_events", None):
         merge_ms = sum(a.elapsed_time(b) for a, b in w.merge_events) / len(w.merge_events)
@@ -723,11 +833,12 @@ def main():
     ap.add_argument("--heads", type=int, default=128,
                     help="heads of the dense workload (128 for the bench line; fewer for profiling)")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "long32k", "chunked", "chunked-context", "sparse",
-                             "sparse-padded"],
+                    choices=["dense", "long32k", "chunked", "chunked-context", "splitkv",
+                             "sparse", "sparse-padded"],
                     help="dense: the headline configuration; long32k: one 32768-token causal "
                          "sequence; chunked: prefix + self passes and the LSE merge; "
-                         "chunked-context: the same in one pass; sparse: the absorbed top-k path")
+                         "chunked-context: the same in one pass; splitkv: a few-tile shape through "
+                         "split-KV; sparse: the absorbed top-k path")
     args = ap.parse_args()
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")

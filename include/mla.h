@@ -206,6 +206,45 @@ int mla_prefill_fwd_ex(const void* q, const void* k, const void* v, const int32_
                        size_t workspace_bytes);
 
 /*
+ * Split-KV (the split-KV path of the "Sgl project Sglang FA4 Interface"
+ * page, Description: num_splits_heuristic and the FlashAttentionForwardCombine
+ * kernel; vLLM's warmup probes of shapes with max_seqlen_q = 1 and long
+ * keys).  When a call has fewer (sequence, 512-row block, head) tiles than
+ * the GPU has CTA pairs, most of them idle; split-KV cuts each tile's KV
+ * blocks into num_splits ranges, computes a partial result (O normalised
+ * over its range, and its LSE) per range into the workspace, and combines
+ * the partials by their LSEs (the N-way form of mla_attn_merge).  The
+ * result equals mla_prefill_fwd's up to floating-point rounding; the split
+ * boundaries depend only on each tile and num_splits, so a call is
+ * deterministic, but its result depends on num_splits (pass 1 where
+ * results must not depend on the batch).
+ */
+#define MLA_MAX_SPLITS 64
+
+/* Workspace bytes of mla_prefill_fwd_splitkv (0 for invalid sizes):
+ * mla_prefill_workspace_size plus num_splits x total_q x num_heads x
+ * (128 + 1) floats of partials.  num_splits == 1 needs no partials. */
+size_t mla_prefill_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_splits);
+
+/* A number of splits for a call of these sizes on the current device (1 when
+ * the call already has a tile for every CTA pair): enough tiles for every
+ * pair, at least two 128-key blocks a split, at most MLA_MAX_SPLITS. */
+int mla_prefill_num_splits(int batch, int total_q, int num_heads, int max_seqlen_q,
+                           int max_seqlen_k);
+
+/* mla_prefill_fwd with num_splits (1 .. MLA_MAX_SPLITS) KV splits per tile
+ * and a workspace of mla_prefill_splitkv_workspace_size bytes.  Enqueues
+ * the planner, the attention kernel and (num_splits > 1) the combine
+ * kernel.  Every other argument is that of mla_prefill_fwd (packed q, k, v).
+ * num_splits == 1 is bit for bit mla_prefill_fwd. */
+int mla_prefill_fwd_splitkv(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            int num_splits, void* out, float* lse, mla_stream_t stream, int batch,
+                            int num_heads, int total_q, int total_k, void* workspace,
+                            size_t workspace_bytes);
+
+/*
  * mla_prefill_fwd for callers that cannot allocate device memory.
  *
  * (The pages have no counterpart to this entry point; it is a convenience of

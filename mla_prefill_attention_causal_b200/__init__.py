@@ -14,7 +14,10 @@ from ._lib import (  # noqa: F401
     mla_prefill_fwd,
     mla_prefill_fwd_context,
     mla_prefill_fwd_ex,
+    mla_prefill_fwd_splitkv,
+    num_splits_for,
     mla_sparse_prefill_fwd,
     prefill_workspace_size,
+    splitkv_workspace_size,
     status_string,
 )

@@ -46,6 +46,10 @@ SIGNATURES = {
                                      _P, _I, _I, _I, _I, _I, _P, _S]),
     "mla_prefill_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _P, _P, _I, _I, _I,
                                 _I, _P, _S]),
+    "mla_prefill_splitkv_workspace_size": (_S, [_I, _I, _I, _I]),
+    "mla_prefill_num_splits": (_I, [_I, _I, _I, _I, _I]),
+    "mla_prefill_fwd_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _I, _P, _P, _P, _I, _I,
+                                     _I, _I, _P, _S]),
     "mla_prefill_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I,
                                      _I]),
     "mla_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
@@ -309,6 +313,57 @@ def mla_prefill_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             _ptr(out), _ptr(lse), _stream(), batch, num_heads, total_q, total_k, _ptr(workspace),
             workspace.numel() * workspace.element_size())
     _check("mla_prefill_fwd_ex", st)
+    return out, lse
+
+
+def num_splits_for(batch: int, total_q: int, num_heads: int, max_seqlen_q: int,
+                   max_seqlen_k: int) -> int:
+    """The library's split-KV choice for these sizes (``mla_prefill_num_splits``)."""
+    return int(load().mla_prefill_num_splits(int(batch), int(total_q), int(num_heads),
+                                             int(max_seqlen_q), int(max_seqlen_k)))
+
+
+def splitkv_workspace_size(batch: int, total_q: int, num_heads: int, num_splits: int) -> int:
+    """Workspace bytes of ``mla_prefill_fwd_splitkv``."""
+    return int(load().mla_prefill_splitkv_workspace_size(int(batch), int(total_q),
+                                                         int(num_heads), int(num_splits)))
+
+
+def mla_prefill_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                            max_seqlen_q: int, max_seqlen_k: int,
+                            softmax_scale: Optional[float] = None, causal: bool = True,
+                            num_splits: Optional[int] = None,
+                            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            return_lse: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Dense prefill with split-KV (``mla_prefill_fwd_splitkv`` in ``mla.h``).
+
+    ``num_splits``: KV splits per tile (1 .. 64), or None for the library's
+    choice (``num_splits_for``).  Packed tensors as ``mla_prefill_fwd``.
+    Returns ``(out [total_q, H, 128] bf16, lse [H, total_q] fp32 or None)``.
+    """
+    batch = cu_seqlens_q.numel() - 1
+    total_q, num_heads = q.shape[0], q.shape[1]
+    if num_splits is None:
+        num_splits = num_splits_for(batch, total_q, num_heads, max_seqlen_q, max_seqlen_k)
+    ws_bytes = splitkv_workspace_size(batch, total_q, num_heads, num_splits)
+    if ws_bytes == 0:
+        raise ValueError(f"invalid split-KV sizes (num_splits={num_splits})")
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    scale, out, lse, workspace, batch, num_heads, total_q, total_k = _packed_dense_args(
+        q, k, v, cu_seqlens_q, cu_seqlens_k, softmax_scale, out, lse, return_lse, workspace)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError(f"workspace must hold >= {ws_bytes} bytes")
+    _same_device(q, k=k, v=v, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, out=out,
+                 lse=lse, workspace=workspace)
+    with torch.cuda.device(q.device):
+        st = load().mla_prefill_fwd_splitkv(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+            int(max_seqlen_k), scale, 1 if causal else 0, int(num_splits), _ptr(out), _ptr(lse),
+            _stream(), batch, num_heads, total_q, total_k, _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    _check("mla_prefill_fwd_splitkv", st)
     return out, lse
 
 

@@ -98,20 +98,23 @@ constexpr int kTileSlots = 4;                        // tiles in flight in the h
 // Workspace layout (caller-provided device memory, 16-byte aligned).
 struct WsHeader {
   int num_entries;  // E: (sequence, 512-row block) entries
-  int num_tiles;    // E * num_heads
+  int num_tiles;    // E * num_heads * nsplit
   int next_tile;    // tiles taken from the counter so far (reset by the planner)
   int pad;
 };
 constexpr size_t kWsHeaderBytes = 256;
 
 // A tile: its sequence's queries, keys and (for a call with a context, see
-// mla_prefill_fwd_context) context keys, the first query row and the head.
-// A tile always has query rows, so Lq == 0 marks "no tile" (the end of a
-// cluster's list).
+// mla_prefill_fwd_context) context keys, the first query row, the head and,
+// for a split-KV call, which of the splits of its KV blocks it covers
+// (packed as hs = head | split << 16).  A tile always has query rows, so
+// Lq == 0 marks "no tile" (the end of a cluster's list).
 struct alignas(16) TileInfo {
   int q_start, Lq, k_start, Lk;
-  int c_start, Lc, m0, h;
+  int c_start, Lc, m0, hs;
   __host__ __device__ bool valid() const { return Lq > 0; }
+  __host__ __device__ int head() const { return hs & 0xffff; }
+  __host__ __device__ int split() const { return hs >> 16; }
 };
 
 struct alignas(16) Bars {
@@ -143,6 +146,9 @@ struct Params {
   float* lse;
   const float* sinks;      // one attention-sink logit per head, or null
   const float* out_scale;  // e4m3 output scale (device scalar), or null: bf16 output
+  float* o_part;           // split-KV: fp32 [nsplit][total_q][H][128] partial outputs
+  float* lse_part;         // split-KV: fp32 [nsplit][H][total_q] partial LSEs
+  int nsplit;              // KV splits per tile (1: none; the partials are unused)
   WsHeader* ws;
   const int2* entries;  // [E] {sequence, 512-row block index}, longest first
   int num_heads;
@@ -174,13 +180,24 @@ __host__ __device__ __forceinline__ int sub_tile_blocks(int row0, int Lq, int Lk
   if (row0 >= Lq) return 0;
   return blocks_for(Lc) + blocks_for(sub_tile_keys(row0, Lq, Lk, causal));
 }
+// Split-KV: a tile's block sequence (nmax = the longer sub-tile's blocks) is
+// cut into nsplit ranges [s nmax / nsplit, (s+1) nmax / nsplit); split s of
+// a sub-tile with n blocks visits blocks [lo, lo + count) of its own.
+__host__ __device__ __forceinline__ int split_lo(int nmax, int s, int nsplit) {
+  return static_cast<int>(static_cast<long long>(nmax) * s / nsplit);
+}
+__host__ __device__ __forceinline__ int split_count(int n, int nmax, int s, int nsplit) {
+  const int lo = split_lo(nmax, s, nsplit), hi = split_lo(nmax, s + 1, nsplit);
+  return max(0, min(hi, n) - lo);
+}
 
 // ------------------------------------------------------------------ planner
 // One CTA: builds the (sequence, 512-row block) entry list sorted by the
 // number of KV blocks its rows visit (descending).
 __global__ void __launch_bounds__(kPlanThreads)
     dense_plan_kernel(const int* cu_q, const int* cu_k, const int* cu_ctx, int batch,
-                      int causal, WsHeader* ws, int2* entries, int capacity, int num_heads) {
+                      int causal, WsHeader* ws, int2* entries, int capacity, int num_heads,
+                      int nsplit) {
   __shared__ int bins[kPlanBins];
   __shared__ int s_total;
   const int tid = threadIdx.x;
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     if (s_total > capacity) atomicOr(&g_mla_status, MLA_DEVSTAT_PLAN_OVERFLOW);
     const int e = min(s_total, capacity);
     ws->num_entries = e;
-    ws->num_tiles = e * num_heads;
+    ws->num_tiles = e * num_heads * nsplit;
     ws->next_tile = 0;
   }
   __syncthreads();
@@ -271,11 +288,14 @@ __device__ __forceinline__ int tail_heads(int num_heads, int num_entries, int nc
 }
 
 // Coordinates of tile t of the list: head-major over the sorted entries,
-// then entry-major over the last `tail` heads (see the file comment).
+// then entry-major over the last `tail` heads (see the file comment); the
+// splits of one (entry, head) are consecutive.
 __device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_tiles,
                                               int num_entries, int tail) {
   TileInfo ti;
   if (t < num_tiles) {
+    const int split = t % p.nsplit;
+    t /= p.nsplit;
     const int H = p.num_heads;
     const int bulk = (H - tail) * num_entries;
     int h, e;
@@ -295,16 +315,23 @@ __device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_ti
     ti.c_start = p.cu_ctx != nullptr ? p.cu_ctx[en.x] : 0;
     ti.Lc = p.cu_ctx != nullptr ? p.cu_ctx[en.x + 1] - ti.c_start : 0;
     ti.m0 = en.y * kTileRows;
-    ti.h = h;
+    ti.hs = h | (split << 16);
   } else {
-    ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.c_start = ti.Lc = ti.m0 = ti.h = 0;
+    ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.c_start = ti.Lc = ti.m0 = ti.hs = 0;
   }
   return ti;
 }
 
-__device__ __forceinline__ void tile_blocks(const TileInfo& t, int causal, int (&n)[2]) {
-  n[0] = sub_tile_blocks(t.m0, t.Lq, t.Lk, t.Lc, causal);
-  n[1] = sub_tile_blocks(t.m0 + kSubRows, t.Lq, t.Lk, t.Lc, causal);
+// KV blocks of the tile's two sub-tiles in its split, and the split's first
+// block.
+__device__ __forceinline__ void tile_blocks(const TileInfo& t, int causal, int nsplit,
+                                            int (&n)[2], int& lo) {
+  const int f0 = sub_tile_blocks(t.m0, t.Lq, t.Lk, t.Lc, causal);
+  const int f1 = sub_tile_blocks(t.m0 + kSubRows, t.Lq, t.Lk, t.Lc, causal);
+  const int nmax = max(f0, f1);
+  lo = split_lo(nmax, t.split(), nsplit);
+  n[0] = split_count(f0, nmax, t.split(), nsplit);
+  n[1] = split_count(f1, nmax, t.split(), nsplit);
 }
 
 __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
@@ -381,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int causal = p.causal;
   const int num_tiles = p.ws->num_tiles;
   const int num_entries = p.ws->num_entries;
-  const int tail = tail_heads(p.num_heads, num_entries, nclusters);
+  const int tail = tail_heads(p.num_heads, num_entries * p.nsplit, nclusters);
   auto wait = [&](uint32_t bar, uint32_t parity, unsigned err) -> bool {
     return mbar_wait_cluster(bar, parity, abort_flag, err, tlim);
   };
@@ -423,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t fb = mapa_shared(smem_u32(&bars->tile_full[ts]), r);
             mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(sizeof(TileInfo)));
             st_async_v4(mapa_shared(a, r), ti.q_start, ti.Lq, ti.k_start, ti.Lk, fb);
-            st_async_v4(mapa_shared(a + 16, r), ti.c_start, ti.Lc, ti.m0, ti.h, fb);
+            st_async_v4(mapa_shared(a + 16, r), ti.c_start, ti.Lc, ti.m0, ti.hs, fb);
           }
         } else {
           if (!(ok = wait(smem_u32(&bars->tile_full[ts]), tile_par(k),
@@ -433,8 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ti.valid()) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
         }
         if (!ti.valid()) break;
-        int nb[2];
-        tile_blocks(ti, causal, nb);
+        int nb[2], lo;
+        tile_blocks(ti, causal, p.nsplit, nb, lo);
+        const int h = ti.head();
         const int nblk = max(nb[0], nb[1]);
         // Q rows of this CTA, once the previous tile's last S MMA has read them.
         for (int i = 0; i < 2 && ok; ++i) {
@@ -455,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_cluster(qbar);
 #pragma unroll
             for (int c = 0; c < kQkChunks; ++c)
-              tma_load_3d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q, 64 * c, ti.h,
+              tma_load_3d_pair(sQ + (i * kQkChunks + c) * kQChunkBytes, &tm_q, 64 * c, h,
                                ti.q_start + ti.m0 + i * kSubRows + static_cast<int>(rank) * kCtaRows,
                                qbar, pol_q);
           } else {
@@ -466,9 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = 0; n < nblk && ok; ++n, ++blk) {
           const int slot = blk % kSlots;
           const uint32_t par = (static_cast<uint32_t>(blk / kSlots) & 1u) ^ 1u;
-          const bool in_ctx = n < nctx;
-          const int key0 = in_ctx ? ti.c_start + n * kBlockKeys
-                                  : ti.k_start + (n - nctx) * kBlockKeys;
+          const int bi = lo + n;  // block of the tile's sequence
+          const bool in_ctx = bi < nctx;
+          const int key0 = in_ctx ? ti.c_start + bi * kBlockKeys
+                                  : ti.k_start + (bi - nctx) * kBlockKeys;
           const CUtensorMap* mk = in_ctx ? &tm_kc : &tm_k;
           const CUtensorMap* mv = in_ctx ? &tm_vc : &tm_v;
           // K: this CTA's 64 keys, three 64-dim chunks of the 192
@@ -480,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kbar = lead(&bars->full_kv[slot]);
 #pragma unroll
           for (int u = 0; u < kKUnits; ++u)
-            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, mk, 64 * u, ti.h,
+            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, mk, 64 * u, h,
                              key0 + static_cast<int>(rank) * kHalfKeys, kbar, pol_kv);
           // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
           if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
@@ -489,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < kVUnits; ++u)
             tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, mv,
-                             static_cast<int>(rank) * kHalfDv, ti.h, key0 + 64 * u, vbar, pol_kv);
+                             static_cast<int>(rank) * kHalfDv, h, key0 + 64 * u, vbar, pol_kv);
         }
       }
       if (!ok && leader) {
@@ -566,10 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto fetch = [&](int k, int& valid, int (&n)[2]) -> bool {
         const int ts = tile_slot(k);
         if (!wait_bar(smem_u32(&bars->tile_full[ts]), tile_par(k))) return false;
-        const TileInfo* t = &bars->tiles[ts];
-        valid = t->valid();
-        n[0] = valid ? sub_tile_blocks(t->m0, t->Lq, t->Lk, t->Lc, causal) : 0;
-        n[1] = valid ? sub_tile_blocks(t->m0 + kSubRows, t->Lq, t->Lk, t->Lc, causal) : 0;
+        const TileInfo ti = bars->tiles[ts];
+        valid = ti.valid();
+        int lo;
+        tile_blocks(ti, causal, p.nsplit, n, lo);
         __syncwarp();
         if (valid && lane == 0) mbar_arrive(smem_u32(&bars->tile_empty[ts]));
         return true;
@@ -677,7 +706,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // that row sees (bottom-right causal: row i sees keys j <= i + Lk - Lq)
       const int row0 = slot->m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows;
       const int diag = row0 + Lk - slot->Lq;
-      const int nb = sub_tile_blocks(slot->m0 + sub * kSubRows, slot->Lq, Lk, Lc, causal);
+      int nb, lo;  // this sub-tile's blocks in the tile's split, from block lo on
+      {
+        int n2[2];
+        tile_blocks(*slot, causal, p.nsplit, n2, lo);
+        nb = n2[sub];
+      }
       const int ldiag = diag + wq * 32 + lane;  // this thread's row's last key
       const int lim = causal ? min(Lk, ldiag + 1) : Lk;  // own keys [0, lim) visible
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazily updated)
@@ -697,8 +731,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Blocks [0, nc) hold context keys 128 n + j, visible below Lc; the
         // sequence's own keys follow, visible below the row's limit.  A block
         // that every row of the CTA sees whole needs no mask.
-        const bool in_ctx = n < nc;
-        const int kbase = (in_ctx ? n : n - nc) * kBlockKeys;
+        const int bi = lo + n;  // block of the tile's sequence
+        const bool in_ctx = bi < nc;
+        const int kbase = (in_ctx ? bi : bi - nc) * kBlockKeys;
         const bool full_blk =
             in_ctx ? kbase + kBlockKeys <= Lc
                    : (kbase + kBlockKeys <= Lk) && (!causal || kbase + kBlockKeys - 1 <= diag);
@@ -759,7 +794,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const int e_lq = bars->tiles[ts].Lq;
       const int e_q0 = bars->tiles[ts].q_start;
-      const int e_h = bars->tiles[ts].h;
+      const int e_h = bars->tiles[ts].head();
+      const int e_split = bars->tiles[ts].split();
       const int r = bars->tiles[ts].m0 + sub * kSubRows + static_cast<int>(rank) * kCtaRows +
                     wq * 32 + lane;  // this thread's row within the sequence
       // Done with the tile's ring slot.  Freed here rather than at the start
@@ -803,7 +839,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             lse2 = mz + lg2_approx(z);
           }
         }
-        if (row_ok && !fp8) {
+        if (row_ok && p.nsplit > 1) {
+          // split-KV: this split's O (normalised by its own sum) in fp32
+          float4* prow = reinterpret_cast<float4*>(
+              p.o_part + (static_cast<size_t>(e_split) * p.total_q * p.num_heads + row_index) * kDv);
+#pragma unroll
+          for (int v4 = 0; v4 < 32; ++v4)
+            prow[v4] = make_float4(__uint_as_float(o[4 * v4]) * scale_o,
+                                   __uint_as_float(o[4 * v4 + 1]) * scale_o,
+                                   __uint_as_float(o[4 * v4 + 2]) * scale_o,
+                                   __uint_as_float(o[4 * v4 + 3]) * scale_o);
+        } else if (row_ok && !fp8) {
           uint4* orow =
               reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_index * kDv);
 #pragma unroll
@@ -831,6 +877,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             orow[v16] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
+      } else if (row_ok && p.nsplit > 1) {
+        // no key of this split: a zero partial with LSE -inf
+        float4* prow = reinterpret_cast<float4*>(
+            p.o_part + (static_cast<size_t>(e_split) * p.total_q * p.num_heads + row_index) * kDv);
+        for (int v = 0; v < 32; ++v) prow[v] = make_float4(0.f, 0.f, 0.f, 0.f);
       } else if (row_ok) {
         // no visible key: zeros (bf16 rows of 256 bytes, e4m3 rows of 128)
         uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
@@ -838,7 +889,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n16 = fp8 ? 8 : 16;
         for (int v = 0; v < n16; ++v) orow[v] = make_uint4(0u, 0u, 0u, 0u);
       }
-      if (row_ok && p.lse != nullptr)
+      if (row_ok && p.nsplit > 1)
+        p.lse_part[(static_cast<size_t>(e_split) * p.num_heads + e_h) * p.total_q + e_q0 + r] =
+            lse2 * 0.69314718055994530942f;
+      else if (row_ok && p.lse != nullptr)
         p.lse[static_cast<size_t>(e_h) * p.total_q + e_q0 + r] = lse2 * 0.69314718055994530942f;
     }
   }

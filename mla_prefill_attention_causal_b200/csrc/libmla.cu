@@ -327,6 +327,7 @@ struct DenseCall {
   int max_ctx = 0, total_ctx = 0;
   const float* sinks = nullptr;
   const float* out_scale = nullptr;
+  int nsplit = 1;  // split-KV: the partials live in the workspace after the work list
   int max_q, max_k;
   float scale;
   int causal;
@@ -337,6 +338,9 @@ struct DenseCall {
   void* workspace;
   size_t workspace_bytes;
 };
+
+// Split-KV partials follow the work list, 256-byte aligned.
+size_t splitkv_parts_offset(size_t work_list_bytes) { return (work_list_bytes + 255) & ~size_t{255}; }
 
 int dense_call(const DenseCall& c) {
   using namespace mla::dense;
@@ -360,11 +364,16 @@ int dense_call(const DenseCall& c) {
               !aligned(c.k_ctx, 16) || !aligned(c.v_ctx, 16) || !aligned(c.cu_ctx, 4) ||
               c.total_ctx < 0 || c.max_ctx < 0))
     return MLA_ERR_INVALID_ARG;
+  if (c.nsplit < 1 || c.nsplit > MLA_MAX_SPLITS || (c.nsplit > 1 && (ctx || c.sinks || c.out_scale)))
+    return MLA_ERR_INVALID_ARG;
   const size_t need = mla_prefill_workspace_size(c.batch, c.total_q);
-  if (c.workspace_bytes < need) return MLA_ERR_INVALID_ARG;
-  // the kernels count tiles (work-list entries x heads, plus one grab per
-  // cluster past the end) in int
-  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * c.num_heads >
+  const size_t need_all =
+      c.nsplit > 1 ? mla_prefill_splitkv_workspace_size(c.batch, c.total_q, c.num_heads, c.nsplit)
+                   : need;
+  if (need_all == 0 || c.workspace_bytes < need_all) return MLA_ERR_INVALID_ARG;
+  // the kernels count tiles (work-list entries x heads x splits, plus one
+  // grab per cluster past the end) in int
+  if (static_cast<long long>((need - kWsHeaderBytes) / sizeof(int2)) * c.num_heads * c.nsplit >
       INT32_MAX - 65536)
     return MLA_ERR_INVALID_ARG;
   int dev = 0;
@@ -398,7 +407,7 @@ int dense_call(const DenseCall& c) {
   int2* entries = reinterpret_cast<int2*>(static_cast<char*>(c.workspace) + kWsHeaderBytes);
   const int capacity = static_cast<int>((need - kWsHeaderBytes) / sizeof(int2));
   dense_plan_kernel<<<1, kPlanThreads, 0, s>>>(c.cu_q, c.cu_k, c.cu_ctx, c.batch, c.causal, ws,
-                                               entries, capacity, c.num_heads);
+                                               entries, capacity, c.num_heads, c.nsplit);
   if ((st = launch_status()) != MLA_OK) return st;
 
   Params p;
@@ -409,6 +418,15 @@ int dense_call(const DenseCall& c) {
   p.lse = c.lse;
   p.sinks = c.sinks;
   p.out_scale = c.out_scale;
+  p.nsplit = c.nsplit;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
+  if (c.nsplit > 1) {
+    char* part = static_cast<char*>(c.workspace) + splitkv_parts_offset(need);
+    p.o_part = reinterpret_cast<float*>(part);
+    p.lse_part = reinterpret_cast<float*>(
+        part + static_cast<size_t>(c.nsplit) * c.total_q * c.num_heads * kDv * sizeof(float));
+  }
   p.ws = ws;
   p.entries = entries;
   p.num_heads = c.num_heads;
@@ -418,7 +436,7 @@ int dense_call(const DenseCall& c) {
   p.timeout_ns = wait_timeout_ns();
   // Persistent: as many 2-CTA clusters as can be resident at once, but never
   // more than tiles could exist.
-  const long long max_tiles = static_cast<long long>(capacity) * c.num_heads;
+  const long long max_tiles = static_cast<long long>(capacity) * c.num_heads * c.nsplit;
   const long long resident = g_dev[dev].dense_clusters.load(std::memory_order_relaxed);
   const long long clusters = max_tiles < resident ? max_tiles : resident;
   cudaLaunchConfig_t cfg = {};
@@ -437,6 +455,16 @@ int dense_call(const DenseCall& c) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }
+  if ((st = launch_status()) != MLA_OK || c.nsplit == 1) return st;
+  // split-KV: combine the partials of every (token, head) row
+  namespace mg = mla::merge;
+  const long long rows = static_cast<long long>(c.total_q) * c.num_heads;
+  const long long warps_per_block = mg::kCombineThreads / 32;
+  const long long want = (rows + warps_per_block - 1) / warps_per_block;
+  const long long cap = static_cast<long long>(g_dev[dev].sms.load(std::memory_order_relaxed)) * 8;
+  mg::combine_splits_kernel<<<static_cast<unsigned>(want < cap ? want : cap), mg::kCombineThreads, 0,
+                              s>>>(reinterpret_cast<const float4*>(p.o_part), p.lse_part, c.nsplit,
+                                   c.total_q, c.num_heads, static_cast<uint2*>(c.out), c.lse);
   return launch_status();
 }
 
@@ -528,6 +556,63 @@ int mla_prefill_fwd_context(const void* q, const void* k, const void* v,
   c.cu_ctx = cu_seqlens_ctx;
   c.max_ctx = max_seqlen_ctx;
   c.total_ctx = total_ctx;
+  c.max_q = max_seqlen_q;
+  c.max_k = max_seqlen_k;
+  c.scale = softmax_scale;
+  c.causal = causal;
+  c.out = out;
+  c.lse = lse;
+  c.stream = stream;
+  c.batch = batch;
+  c.num_heads = num_heads;
+  c.total_q = total_q;
+  c.total_k = total_k;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  return dense_call(c);
+}
+
+size_t mla_prefill_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_splits) {
+  const size_t base = mla_prefill_workspace_size(batch, total_q);
+  if (base == 0 || num_heads < 1 || num_splits < 1 || num_splits > MLA_MAX_SPLITS) return 0;
+  if (num_splits == 1) return base;
+  const size_t rows = static_cast<size_t>(total_q) * static_cast<size_t>(num_heads);
+  return splitkv_parts_offset(base) +
+         static_cast<size_t>(num_splits) * rows * (mla::dense::kDv + 1) * sizeof(float);
+}
+
+int mla_prefill_num_splits(int batch, int total_q, int num_heads, int max_seqlen_q,
+                           int max_seqlen_k) {
+  if (batch < 1 || total_q < 0 || num_heads < 1 || max_seqlen_q < 0 || max_seqlen_k < 0) return 1;
+  using mla::dense::kBlockKeys;
+  using mla::dense::kTileRows;
+  int dev = 0;
+  int clusters = 74;  // the B200's 148 SMs as CTA pairs, if no device is current
+  if (prepare_device(&dev) == MLA_OK)
+    clusters = g_dev[dev].dense_clusters.load(std::memory_order_relaxed);
+  // tiles the call has at most: (sequence, 512-row block) entries x heads
+  const long long per_seq = (static_cast<long long>(max_seqlen_q) + kTileRows - 1) / kTileRows;
+  const long long by_total = (static_cast<long long>(total_q) + kTileRows - 1) / kTileRows + batch;
+  const long long entries = per_seq * batch < by_total ? per_seq * batch : by_total;
+  const long long tiles = entries * num_heads;
+  if (tiles <= 0 || tiles >= clusters) return 1;
+  long long n = (clusters + tiles - 1) / tiles;               // enough tiles for every cluster
+  const long long blocks = (static_cast<long long>(max_seqlen_k) + kBlockKeys - 1) / kBlockKeys;
+  if (n > blocks / 2) n = blocks / 2;                         // at least two KV blocks a split
+  if (n > MLA_MAX_SPLITS) n = MLA_MAX_SPLITS;
+  return n < 1 ? 1 : static_cast<int>(n);
+}
+
+int mla_prefill_fwd_splitkv(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                            int num_splits, void* out, float* lse, mla_stream_t stream, int batch,
+                            int num_heads, int total_q, int total_k, void* workspace,
+                            size_t workspace_bytes) {
+  DenseCall c = packed_call(q, k, v, num_heads);
+  c.cu_q = cu_seqlens_q;
+  c.cu_k = cu_seqlens_k;
+  c.nsplit = num_splits;
   c.max_q = max_seqlen_q;
   c.max_k = max_seqlen_k;
   c.scale = softmax_scale;

@@ -96,3 +96,54 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace merge
 }  // namespace mla
+
+namespace mla {
+namespace merge {
+
+// Split-KV combine: the N-way form of the merge above (the combine step of
+// the split-KV path the FA4 interface page describes, and of the Mojo mla
+// module's mla_splitk_reduce).  For each (token, head) row with partial
+// results (O_s, lse_s), s < nsplit, over disjoint key ranges:
+//   lse = m + ln sum_s e^(lse_s - m),  m = max_s lse_s
+//   out = sum_s e^(lse_s - lse) O_s
+// A split without keys has lse_s = -inf (weight 0); a row without any key
+// gets out = 0, lse = -inf.  Partials: o_part fp32 [nsplit][T][H][128],
+// lse_part [nsplit][H][T]; out bf16 [T][H][128], lse [H][T] (may be null).
+// One warp per row, four dims per lane.
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_splits_kernel(const float4* __restrict__ o_part, const float* __restrict__ lse_part,
+                          int nsplit, int num_tokens, int num_heads, uint2* out, float* lse) {
+  const long long rows = static_cast<long long>(num_tokens) * num_heads;
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < rows; row += warps) {
+    const int t = static_cast<int>(row / num_heads), h = static_cast<int>(row % num_heads);
+    const size_t li = static_cast<size_t>(h) * num_tokens + t;
+    const size_t split_lse = static_cast<size_t>(num_heads) * num_tokens;
+    float m = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) m = fmaxf(m, lse_part[s * split_lse + li]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float z = 0.f;
+    if (m != -INFINITY) {
+      for (int s = 0; s < nsplit; ++s) {
+        const float w = exp2f((lse_part[s * split_lse + li] - m) * 1.4426950408889634f);
+        const float4 o = o_part[(static_cast<size_t>(s) * rows + row) * 32 + lane];
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+        z += w;
+      }
+    }
+    const float inv = z > 0.f ? 1.0f / z : 0.f;
+    out[row * 32 + lane] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
+                                      pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (lse != nullptr && lane == 0) lse[li] = z > 0.f ? m + logf(z) : -INFINITY;
+  }
+}
+
+}  // namespace merge
+}  // namespace mla

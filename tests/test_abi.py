@@ -197,3 +197,35 @@ def _call_ex(**over):
                                   dict(scale=0.0), dict(H=0)])
 def test_ex_call_rejects_bad_arguments(over):
     assert _call_ex(**over) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_splitkv_sizes_and_choice():
+    f = mla.splitkv_workspace_size
+    base = mla.prefill_workspace_size(2, 100)
+    assert f(2, 100, 8, 1) == base                       # no partials without splits
+    parts = ((base + 255) // 256) * 256
+    assert f(2, 100, 8, 3) == parts + 3 * 100 * 8 * 129 * 4
+    assert f(2, 100, 8, 0) == 0 and f(2, 100, 8, 65) == 0 and f(2, 100, 0, 2) == 0
+    # no GPU here: the choice assumes 74 CTA pairs
+    assert mla.num_splits_for(1, 1, 16, 1, 8192) == 5     # 16 tiles -> ceil(74/16)
+    assert mla.num_splits_for(1, 1, 128, 1, 8192) == 1    # a tile for every pair already
+    assert mla.num_splits_for(1, 1, 4, 1, 512) == 2       # at least two KV blocks a split
+    assert mla.num_splits_for(1, 1, 1, 1, 1 << 20) == 64  # at most MLA_MAX_SPLITS
+    assert mla.num_splits_for(8, 16384, 128, 4096, 4096) == 1
+
+
+def _call_split(**over):
+    a = dict(q=16, k=16, v=16, cq=16, ck=16, mq=4, mk=4, scale=0.1, causal=1, ns=2, out=16,
+             lse=None, batch=1, H=1, tq=4, tk=4, ws=64, wsb=1 << 20)
+    a.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return mla.load().mla_prefill_fwd_splitkv(
+        P(a["q"]), P(a["k"]), P(a["v"]), P(a["cq"]), P(a["ck"]), a["mq"], a["mk"], a["scale"],
+        a["causal"], a["ns"], P(a["out"]), P(a["lse"]), None, a["batch"], a["H"], a["tq"],
+        a["tk"], P(a["ws"]), a["wsb"])
+
+
+@pytest.mark.parametrize("over", [dict(ns=0), dict(ns=65), dict(wsb=300), dict(q=None),
+                                  dict(out=8), dict(causal=2)])
+def test_splitkv_call_rejects_bad_arguments(over):
+    assert _call_split(**over) == _lib.MLA_ERR_INVALID_ARG

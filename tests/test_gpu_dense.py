@@ -368,3 +368,62 @@ def test_sinks_with_fp8_output():
     got = oracle.e4m3_decode(out.view(torch.uint8).cpu().numpy())
     y_b = np.clip(to_f64(o_b) / 0.02, -448.0, 448.0)
     assert np.all(np.abs(got - y_b) <= _e4m3_step(y_b) * 1.0001)
+
+
+# -------------------------------------------------------------------- split-KV
+def _run_split(case, num_splits):
+    import mla_prefill_attention_causal_b200 as mla
+    out, lse = mla.mla_prefill_fwd_splitkv(
+        dev_bf16(case["q"]), dev_bf16(case["k"]), dev_bf16(case["v"]), dev_i32(case["cu_q"]),
+        dev_i32(case["cu_k"]), case["max_q"], case["max_k"], case["scale"], causal=case["causal"],
+        num_splits=num_splits)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+@pytest.mark.parametrize("max_q,max_k", [(1, 4096), (1, 8192), (129, 4096), (129, 512)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_splitkv_on_the_warmup_probe_shapes(max_q, max_k, causal):
+    """vLLM's MLA warmup probes with few heads (a tensor-parallel share):
+    fewer tiles than CTA pairs, so the library splits the KV blocks."""
+    import mla_prefill_attention_causal_b200 as mla
+    case = syn.dense_case([max_q], [max_k], 4, seed=max_q + max_k + 7, causal=causal)
+    ns = mla.num_splits_for(1, max_q, 4, max_q, max_k)
+    assert ns > 1
+    out, lse = _run_split(case, None)
+    ref_o, ref_l = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"],
+                                        case["cu_k"], case["scale"], causal)
+    assert_out_close(to_f64(out), ref_o, f"split-KV ({ns} splits) out")
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), ref_l, f"split-KV ({ns} splits) lse")
+
+
+@pytest.mark.parametrize("splits", [2, 3, 7, 64])
+def test_splitkv_ragged_batch(splits):
+    """A ragged causal batch with rows without keys (Lq > Lk) and an empty
+    key sequence; 64 splits leave most ranges of the short tiles empty."""
+    lens_q = [300, 129, 1, 200, 40]
+    lens_k = [900, 129, 700, 150, 0]
+    case = syn.dense_case(lens_q, lens_k, 2, seed=101 + splits, causal=True)
+    out, lse = _run_split(case, splits)
+    ref_o, ref_l = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"],
+                                        case["cu_k"], case["scale"], True)
+    assert_out_close(to_f64(out), ref_o, "split-KV ragged out")
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), ref_l, "split-KV ragged lse")
+    assert np.all(to_f64(out)[sum(lens_q[:4]):] == 0)
+
+
+def test_splitkv_with_one_split_is_the_plain_call():
+    case = syn.dense_case([700, 129, 1300], [700, 129, 1300], 4, seed=102)
+    o, l = _run_split(case, 1)
+    o_p, l_p = run_dense(case)
+    assert torch.equal(o, o_p) and torch.equal(l, l_p)
+
+
+def test_splitkv_is_deterministic_and_close_to_unsplit():
+    case = syn.dense_case([1], [8192], 8, seed=103, causal=False)
+    a, la = _run_split(case, 9)
+    b, lb = _run_split(case, 9)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+    o_p, l_p = run_dense(case)
+    assert (a.float() - o_p.float()).abs().max().item() <= 2 ** -7
+    assert (la - l_p).abs().max().item() <= 1e-4

@@ -381,7 +381,7 @@ class ChunkedWorkload:
               "(causal-adj) and % of B200 dense BF16 peak, 1 GPU")
     kernel = "mla::dense::dense_fwd_kernel"
     sources = ("dense_fwd.cuh", "ptx.cuh")
-    profile = "dense_fwd_varlen16k.md"
+    profile = "dense_fwd_chunked.md"  # DRAM bytes of the step's two attention launches
     merge_sources = ("merge.cuh",)
     merge_profile = "merge_chunked.md"
     data = "synthetic (seeded N(0,1) bf16 query chunks, prefix and self K/V)"

@@ -245,6 +245,26 @@ int mla_prefill_fwd_splitkv(const void* q, const void* k, const void* v,
                             size_t workspace_bytes);
 
 /*
+ * mla_prefill_fwd for the other MLA head geometries of vLLM's MLA prefill
+ * backend ("flash_attn.py", supports_mla_dimensions: (qk_nope, qk_rope, v)
+ * = (128, 64, 128), (192, 64, 256), (64, 64, 128) and (256, 0, 256)):
+ * qk_dim = qk_nope + qk_rope in {128, 192, 256}, v_dim in {128, 256}.
+ *   q [total_q, H, qk_dim], k [total_k, H, qk_dim], v [total_k, H, v_dim],
+ *   out [total_q, H, v_dim] (bf16, packed, 16-B aligned); lse as in
+ *   mla_prefill_fwd.
+ * The kernel computes 128 value dims per pass: v_dim = 256 runs two passes
+ * over the halves of V (strided views), each recomputing the scores, and
+ * writes the LSE in the first.  (qk_dim, v_dim) = (192, 128) is
+ * mla_prefill_fwd.  Same workspace as mla_prefill_fwd.
+ */
+int mla_prefill_fwd_dims(const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                         int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                         void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                         int total_q, int total_k, int qk_dim, int v_dim, void* workspace,
+                         size_t workspace_bytes);
+
+/*
  * mla_prefill_fwd for callers that cannot allocate device memory.
  *
  * (The pages have no counterpart to this entry point; it is a convenience of

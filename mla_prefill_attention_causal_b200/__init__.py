@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     mla_device_status,
     mla_prefill_fwd,
     mla_prefill_fwd_context,
+    mla_prefill_fwd_dims,
     mla_prefill_fwd_ex,
     mla_prefill_fwd_splitkv,
     num_splits_for,

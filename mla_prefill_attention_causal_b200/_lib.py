@@ -46,6 +46,8 @@ SIGNATURES = {
                                      _P, _I, _I, _I, _I, _I, _P, _S]),
     "mla_prefill_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _P, _P, _I, _I, _I,
                                 _I, _P, _S]),
+    "mla_prefill_fwd_dims": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _P, _P, _P, _I, _I, _I, _I,
+                                  _I, _I, _P, _S]),
     "mla_prefill_splitkv_workspace_size": (_S, [_I, _I, _I, _I]),
     "mla_prefill_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "mla_prefill_fwd_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _F, _I, _I, _P, _P, _P, _I, _I,
@@ -313,6 +315,62 @@ def mla_prefill_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             _ptr(out), _ptr(lse), _stream(), batch, num_heads, total_q, total_k, _ptr(workspace),
             workspace.numel() * workspace.element_size())
     _check("mla_prefill_fwd_ex", st)
+    return out, lse
+
+
+def mla_prefill_fwd_dims(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                         max_seqlen_q: int, max_seqlen_k: int,
+                         softmax_scale: Optional[float] = None, causal: bool = True,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         return_lse: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Dense prefill for the other MLA head geometries (``mla_prefill_fwd_dims``).
+
+    q/k ``[*, H, qk_dim]`` with qk_dim in {128, 192, 256}, v ``[*, H, v_dim]``
+    with v_dim in {128, 256}; packed bf16.  Returns ``(out [total_q, H,
+    v_dim] bf16, lse [H, total_q] fp32 or None)``.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, num_heads, qk_dim = q.shape
+    total_k, v_dim = k.shape[0], v.shape[2]
+    if qk_dim not in (128, 192, 256) or v_dim not in (128, 256):
+        raise ValueError(f"unsupported MLA dims: qk {qk_dim}, v {v_dim}")
+    if k.shape[1:] != (num_heads, qk_dim) or v.shape[:2] != (total_k, num_heads):
+        raise ValueError("q, k and v must agree on heads and dims, k and v on rows")
+    batch = cu_seqlens_q.numel() - 1
+    if batch < 1 or cu_seqlens_k.numel() != batch + 1:
+        raise ValueError("cu_seqlens_q/k must both have batch+1 >= 2 entries")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(qk_dim)
+    if out is None:
+        out = torch.empty((total_q, num_heads, v_dim), dtype=torch.bfloat16, device=q.device)
+    else:
+        _need(out, "out", torch.bfloat16, 3)
+        if out.shape != (total_q, num_heads, v_dim):
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((num_heads, total_q), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+        if lse.shape != (num_heads, total_q):
+            raise ValueError("lse must be [num_heads, total_q]")
+    ws_bytes = prefill_workspace_size(batch, total_q)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < ws_bytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of >= {ws_bytes} bytes")
+    _same_device(q, k=k, v=v, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, out=out,
+                 lse=lse, workspace=workspace)
+    with torch.cuda.device(q.device):
+        st = load().mla_prefill_fwd_dims(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+            int(max_seqlen_k), float(softmax_scale), 1 if causal else 0, _ptr(out), _ptr(lse),
+            _stream(), batch, num_heads, total_q, total_k, qk_dim, v_dim, _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    _check("mla_prefill_fwd_dims", st)
     return out, lse
 
 

@@ -66,20 +66,13 @@ constexpr int kSubRows = 256;                        // MMA M (rows per sub-tile
 constexpr int kTileRows = 512;                       // query rows per tile
 constexpr int kBlockKeys = 128;                      // keys per KV block (MMA N of S)
 constexpr int kHalfKeys = 64;                        // keys of a K block held by one CTA
-constexpr int kDqk = 192;
-constexpr int kDv = 128;
+constexpr int kDqk = 192;                            // qk width of the MLA dims 128 + 64
+constexpr int kDv = 128;                             // value dims of one pass
 constexpr int kHalfDv = 64;                          // value dims held by one CTA
 constexpr int kQChunkBytes = 128 * 128;              // 128 rows x 64 bf16
 constexpr int kUnitBytes = 64 * 128;                 // 64 rows x 64 bf16
-constexpr int kQkChunks = kDqk / 64;                 // 3
-constexpr int kKUnits = kQkChunks;                   // K half: 64 keys x 192 dims
 constexpr int kVUnits = kBlockKeys / 64;             // V half: 128 keys x 64 dims
-constexpr int kSlots = 3;                            // K and V blocks in flight per CTA
-constexpr int kKSlotBytes = kKUnits * kUnitBytes;    // 24 KB: this CTA's half of a K block
 constexpr int kVSlotBytes = kVUnits * kUnitBytes;    // 16 KB: this CTA's half of a V block
-constexpr int kQSubBytes = kQkChunks * kQChunkBytes; // 48 KB
-constexpr int kQBytes = 2 * kQSubBytes;              // 96 KB
-constexpr int kRingBytes = kSlots * (kKSlotBytes + kVSlotBytes);  // 120 KB
 constexpr int kThreads = 384;          // 3 warpgroups; warps 10-11 only hold registers
 // Register split (setmaxnreg): launched at kLaunchRegs per thread, the two
 // softmax warpgroups grow to kSoftmaxRegs and the producer/MMA warpgroup
@@ -117,6 +110,7 @@ struct alignas(16) TileInfo {
   __host__ __device__ int split() const { return hs >> 16; }
 };
 
+template <int SLOTS>
 struct alignas(16) Bars {
   TileInfo tiles[kTileSlots];     // both: tile hand-off ring (written by the leader's producer)
   static_assert(sizeof(TileInfo) == 32, "a ring slot is two 16-byte stores");
@@ -124,9 +118,9 @@ struct alignas(16) Bars {
   uint64_t tile_empty[kTileSlots];  // leader: every reader of the slot is done with it
   uint64_t q_full[2];    // leader: both producers (and the Q bytes of both CTAs)
   uint64_t q_empty[2];   // both: last S MMA of the tile done
-  uint64_t full_kv[kSlots];  // leader: K- and V-half bytes of block b, both CTAs
-  uint64_t empty_k[kSlots];  // both: the S MMAs reading the K slot done
-  uint64_t empty_v[kSlots];  // both: the PV MMAs reading the V slot done
+  uint64_t full_kv[SLOTS];   // leader: K- and V-half bytes of block b, both CTAs
+  uint64_t empty_k[SLOTS];   // both: the S MMAs reading the K slot done
+  uint64_t empty_v[SLOTS];   // both: the PV MMAs reading the V slot done
   uint64_t s_full[2];    // both
   uint64_t p_full[2];    // leader: 8 softmax warps (both CTAs)
   uint64_t o_full[2];    // both
@@ -136,13 +130,32 @@ struct alignas(16) Bars {
   int abort;
 };
 
-constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + static_cast<int>(sizeof(Bars));
+// Shared-memory plan for a qk width of DQK (128, 192 or 256) dims: Q of both
+// sub-tiles (DQK/64 chunks of 128 rows x 64 dims each) and a ring of K/V
+// block halves -- three slots, or two at DQK = 256, where Q alone takes
+// 128 KB.  The value width of one pass is always 128 (kDv).
+template <int DQK>
+struct Geo {
+  static_assert(DQK == 128 || DQK == 192 || DQK == 256, "qk width");
+  static constexpr int kQkChunks = DQK / 64;
+  static constexpr int kKUnits = kQkChunks;                   // K half: 64 keys x DQK dims
+  static constexpr int kSlots = DQK == 256 ? 2 : 3;           // K and V blocks in flight
+  static constexpr int kKSlotBytes = kKUnits * kUnitBytes;    // this CTA's half of a K block
+  static constexpr int kQSubBytes = kQkChunks * kQChunkBytes;
+  static constexpr int kQBytes = 2 * kQSubBytes;
+  static constexpr int kRingBytes = kSlots * (kKSlotBytes + kVSlotBytes);
+  static constexpr int kSmemBytes =
+      1024 + kQBytes + kRingBytes + static_cast<int>(sizeof(Bars<kSlots>));
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory above the per-CTA limit");
+};
 
 struct Params {
   const int* cu_q;
   const int* cu_k;
   const int* cu_ctx;       // context keys per sequence ([batch + 1]), or null: no context
   void* out;               // bf16 [total_q, H, 128], or e4m3 when out_scale is set
+  long long out_rs;        // row and head strides of out in elements (H * 128 and 128 for a
+  long long out_hs;        // packed output; wider for one 128-dim pass of a wider value)
   float* lse;
   const float* sinks;      // one attention-sink logit per head, or null
   const float* out_scale;  // e4m3 output scale (device scalar), or null: bf16 output
@@ -346,12 +359,22 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
   tmem_wait_st();
 }
 
+template <int DQK>
 __global__ void __launch_bounds__(kThreads, 1)
     dense_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_kc,
                      const __grid_constant__ CUtensorMap tm_vc, const Params p) {
+  using G = Geo<DQK>;
+  constexpr int kQkChunks = G::kQkChunks;
+  constexpr int kKUnits = G::kKUnits;
+  constexpr int kSlots = G::kSlots;
+  constexpr int kKSlotBytes = G::kKSlotBytes;
+  constexpr int kQSubBytes = G::kQSubBytes;
+  constexpr int kQBytes = G::kQBytes;
+  constexpr int kRingBytes = G::kRingBytes;
+  using BarsT = Bars<kSlots>;
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -363,9 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sQ = smem_u32(base);
-  const uint32_t sRingK = sQ + kQBytes;                  // kSlots x 24 KB
+  const uint32_t sRingK = sQ + kQBytes;                  // kSlots x kKSlotBytes
   const uint32_t sRingV = sRingK + kSlots * kKSlotBytes;  // kSlots x 16 KB
-  Bars* bars = reinterpret_cast<Bars*>(base + kQBytes + kRingBytes);
+  BarsT* bars = reinterpret_cast<BarsT*>(base + kQBytes + kRingBytes);
   volatile int* abort_flag = &bars->abort;
   // the leader CTA's copy of a barrier (cluster address)
   auto lead = [&](uint64_t* bar) -> uint32_t { return mapa_shared(smem_u32(bar), 0); };
@@ -812,6 +835,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // path): output 0, LSE -inf, or the sink's logit.
       const bool row_ok = r < e_lq;
       const size_t row_index = static_cast<size_t>(e_q0 + r) * p.num_heads + e_h;
+      const size_t out_off = static_cast<size_t>(e_q0 + r) * p.out_rs +
+                             static_cast<size_t>(e_h) * p.out_hs;  // first element of the row
       const bool fp8 = p.out_scale != nullptr;
       const float sink2 = p.sinks != nullptr ? p.sinks[e_h] * 1.4426950408889634f : -INFINITY;
       float lse2 = sink2;  // log2 of the row's denominator
@@ -850,8 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    __uint_as_float(o[4 * v4 + 2]) * scale_o,
                                    __uint_as_float(o[4 * v4 + 3]) * scale_o);
         } else if (row_ok && !fp8) {
-          uint4* orow =
-              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_index * kDv);
+          uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + out_off);
 #pragma unroll
           for (int v4 = 0; v4 < 16; ++v4) {
             uint32_t pk[4];
@@ -864,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (row_ok) {
           // e4m3 of O / out_scale: round to nearest even, saturated at 448
           const float qs = scale_o / *p.out_scale;
-          uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row_index * kDv);
+          uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + out_off);
 #pragma unroll
           for (int v16 = 0; v16 < 8; ++v16) {
             uint32_t pk[4];
@@ -885,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (row_ok) {
         // no visible key: zeros (bf16 rows of 256 bytes, e4m3 rows of 128)
         uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
-                                               row_index * kDv * (fp8 ? 1 : 2));
+                                               out_off * (fp8 ? 1 : 2));
         const int n16 = fp8 ? 8 : 16;
         for (int v = 0; v < n16; ++v) orow[v] = make_uint4(0u, 0u, 0u, 0u);
       }

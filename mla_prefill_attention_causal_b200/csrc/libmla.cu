@@ -106,19 +106,25 @@ int setup_device(int dev, int* status, int* sms, int* clusters) {
     *status = MLA_ERR_UNSUPPORTED;
     return MLA_OK;
   }
-  if (cudaFuncSetAttribute(mla::dense::dense_fwd_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           mla::dense::kSmemBytes) != cudaSuccess)
-    return MLA_ERR_CUDA;
   {
-    // The kernel's setmaxnreg split assumes this launch register count; a
-    // different count could make the warps that grow wait for ever.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, mla::dense::dense_fwd_kernel) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    if (fa.numRegs != mla::dense::kLaunchRegs) {
-      *status = MLA_ERR_UNSUPPORTED;
-      return MLA_OK;
+    // Every qk width's kernel: its shared memory, and the launch register
+    // count its setmaxnreg split assumes (a different count could make the
+    // warps that grow wait for ever).
+    const void* kernels[3] = {reinterpret_cast<const void*>(mla::dense::dense_fwd_kernel<128>),
+                              reinterpret_cast<const void*>(mla::dense::dense_fwd_kernel<192>),
+                              reinterpret_cast<const void*>(mla::dense::dense_fwd_kernel<256>)};
+    const int smem[3] = {mla::dense::Geo<128>::kSmemBytes, mla::dense::Geo<192>::kSmemBytes,
+                         mla::dense::Geo<256>::kSmemBytes};
+    for (int i = 0; i < 3; ++i) {
+      if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem[i]) != cudaSuccess)
+        return MLA_ERR_CUDA;
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kernels[i]) != cudaSuccess) return MLA_ERR_CUDA;
+      if (fa.numRegs != mla::dense::kLaunchRegs) {
+        *status = MLA_ERR_UNSUPPORTED;
+        return MLA_OK;
+      }
     }
   }
   if (cudaFuncSetAttribute(mla::sparse::sparse_fwd_kernel,
@@ -137,10 +143,10 @@ int setup_device(int dev, int* status, int* sms, int* clusters) {
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * (*sms / 2), 1, 1);
     cfg.blockDim = dim3(mla::dense::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = mla::dense::kSmemBytes;
+    cfg.dynamicSmemBytes = mla::dense::Geo<256>::kSmemBytes;  // the largest of the three
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(clusters, mla::dense::dense_fwd_kernel, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(clusters, mla::dense::dense_fwd_kernel<256>, &cfg) !=
             cudaSuccess ||
         *clusters < 1)
       return MLA_ERR_CUDA;
@@ -328,6 +334,8 @@ struct DenseCall {
   const float* sinks = nullptr;
   const float* out_scale = nullptr;
   int nsplit = 1;  // split-KV: the partials live in the workspace after the work list
+  int qk_dim = mla::dense::kDqk;  // 128, 192 or 256
+  long long out_rs = 0, out_hs = 0;  // output strides in elements (0: packed [T, H, 128])
   int max_q, max_k;
   float scale;
   int causal;
@@ -356,6 +364,7 @@ int dense_call(const DenseCall& c) {
       c.max_q < 0 || c.max_k < 0 || (c.causal != 0 && c.causal != 1))
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(c.scale) || !(c.scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  if (c.qk_dim != 128 && c.qk_dim != 192 && c.qk_dim != 256) return MLA_ERR_INVALID_ARG;
   if (!good_stride(c.q_rs) || !good_stride(c.q_hs) || !good_stride(c.k_rs) ||
       !good_stride(c.k_hs) || !good_stride(c.v_rs) || !good_stride(c.v_hs))
     return MLA_ERR_INVALID_ARG;
@@ -384,16 +393,17 @@ int dense_call(const DenseCall& c) {
   CUtensorMap tq, tk, tv, tkc, tvc;
   const uint64_t kv_rows = c.total_k > 0 ? static_cast<uint64_t>(c.total_k) : 1;
   const uint64_t H = static_cast<uint64_t>(c.num_heads);
-  if ((st = encode_heads(&tq, c.q, kDqk, H, static_cast<uint64_t>(c.total_q), c.q_hs, c.q_rs,
+  const uint64_t dqk = static_cast<uint64_t>(c.qk_dim);
+  if ((st = encode_heads(&tq, c.q, dqk, H, static_cast<uint64_t>(c.total_q), c.q_hs, c.q_rs,
                          kCtaRows)) != MLA_OK ||
-      (st = encode_heads(&tk, c.k, kDqk, H, kv_rows, c.k_hs, c.k_rs, kHalfKeys)) != MLA_OK ||
+      (st = encode_heads(&tk, c.k, dqk, H, kv_rows, c.k_hs, c.k_rs, kHalfKeys)) != MLA_OK ||
       (st = encode_heads(&tv, c.v, kDv, H, kv_rows, c.v_hs, c.v_rs, 64)) != MLA_OK)
     return st;
   if (ctx) {
     // the context is packed: [total_ctx, H, 192] and [total_ctx, H, 128]
     const uint64_t c_rows = c.total_ctx > 0 ? static_cast<uint64_t>(c.total_ctx) : 1;
     const int64_t hs = c.num_heads;
-    if ((st = encode_heads(&tkc, c.k_ctx, kDqk, H, c_rows, kDqk, hs * kDqk, kHalfKeys)) !=
+    if ((st = encode_heads(&tkc, c.k_ctx, dqk, H, c_rows, c.qk_dim, hs * c.qk_dim, kHalfKeys)) !=
             MLA_OK ||
         (st = encode_heads(&tvc, c.v_ctx, kDv, H, c_rows, kDv, hs * kDv, 64)) != MLA_OK)
       return st;
@@ -415,6 +425,8 @@ int dense_call(const DenseCall& c) {
   p.cu_k = c.cu_k;
   p.cu_ctx = c.cu_ctx;
   p.out = c.out;
+  p.out_rs = c.out_rs != 0 ? c.out_rs : static_cast<long long>(c.num_heads) * kDv;
+  p.out_hs = c.out_hs != 0 ? c.out_hs : kDv;
   p.lse = c.lse;
   p.sinks = c.sinks;
   p.out_scale = c.out_scale;
@@ -447,11 +459,21 @@ int dense_call(const DenseCall& c) {
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, dense_fwd_kernel, tq, tk, tv, tkc, tvc, p) != cudaSuccess) {
+  cudaError_t le;
+  if (c.qk_dim == 192) {
+    cfg.dynamicSmemBytes = Geo<192>::kSmemBytes;
+    le = cudaLaunchKernelEx(&cfg, dense_fwd_kernel<192>, tq, tk, tv, tkc, tvc, p);
+  } else if (c.qk_dim == 256) {
+    cfg.dynamicSmemBytes = Geo<256>::kSmemBytes;
+    le = cudaLaunchKernelEx(&cfg, dense_fwd_kernel<256>, tq, tk, tv, tkc, tvc, p);
+  } else {
+    cfg.dynamicSmemBytes = Geo<128>::kSmemBytes;
+    le = cudaLaunchKernelEx(&cfg, dense_fwd_kernel<128>, tq, tk, tv, tkc, tvc, p);
+  }
+  if (le != cudaSuccess) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }
@@ -627,6 +649,56 @@ int mla_prefill_fwd_splitkv(const void* q, const void* k, const void* v,
   c.workspace = workspace;
   c.workspace_bytes = workspace_bytes;
   return dense_call(c);
+}
+
+int mla_prefill_fwd_dims(const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                         int max_seqlen_q, int max_seqlen_k, float softmax_scale, int causal,
+                         void* out, float* lse, mla_stream_t stream, int batch, int num_heads,
+                         int total_q, int total_k, int qk_dim, int v_dim, void* workspace,
+                         size_t workspace_bytes) {
+  using mla::dense::kDv;
+  if ((qk_dim != 128 && qk_dim != 192 && qk_dim != 256) || (v_dim != 128 && v_dim != 256) ||
+      num_heads < 1)
+    return MLA_ERR_INVALID_ARG;
+  // One pass per 128 value dims: pass j reads v[..., 128 j : 128 j + 128] and
+  // writes out[..., 128 j : 128 j + 128] (strided views); the scores, and so
+  // the LSE, are the same in every pass, which writes it only in the first.
+  const int passes = v_dim / kDv;
+  const int64_t H = num_heads;
+  for (int j = 0; j < passes; ++j) {
+    DenseCall c;
+    c.q = q;
+    c.q_rs = H * qk_dim;
+    c.q_hs = qk_dim;
+    c.k = k;
+    c.k_rs = H * qk_dim;
+    c.k_hs = qk_dim;
+    c.v = v == nullptr ? nullptr : static_cast<const char*>(v) + static_cast<size_t>(j) * kDv * 2;
+    c.v_rs = H * v_dim;
+    c.v_hs = v_dim;
+    c.qk_dim = qk_dim;
+    c.out = out == nullptr ? nullptr : static_cast<char*>(out) + static_cast<size_t>(j) * kDv * 2;
+    c.out_rs = H * v_dim;
+    c.out_hs = v_dim;
+    c.cu_q = cu_seqlens_q;
+    c.cu_k = cu_seqlens_k;
+    c.max_q = max_seqlen_q;
+    c.max_k = max_seqlen_k;
+    c.scale = softmax_scale;
+    c.causal = causal;
+    c.lse = j == 0 ? lse : nullptr;
+    c.stream = stream;
+    c.batch = batch;
+    c.num_heads = num_heads;
+    c.total_q = total_q;
+    c.total_k = total_k;
+    c.workspace = workspace;
+    c.workspace_bytes = workspace_bytes;
+    const int st = dense_call(c);
+    if (st != MLA_OK) return st;
+  }
+  return MLA_OK;
 }
 
 int mla_prefill_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,

@@ -25,7 +25,7 @@ from __future__ import annotations
 
 import random
 
-SLOTS = 3        # K and V ring slots
+SLOTS = 3        # K and V ring slots (two at the 256-wide qk geometry)
 TILE_SLOTS = 4   # tile hand-off ring
 Q_BYTES = 2      # transaction units: Q of a sub-tile per CTA
 KV_BYTES = 2     # K + V half of a block per CTA
@@ -84,13 +84,14 @@ class Model:
     """One CTA pair working through `tiles`, a list of (n0, n1) KV block counts."""
 
     def __init__(self, tiles, rng: random.Random, q_full_both: bool = True,
-                 early_fetch: bool = False):
+                 early_fetch: bool = False, slots: int = SLOTS):
         # The two switches restate designs the kernel does not use, for the
         # test that shows the model catches them: q_full_both=False lets only
         # the leader's producer arrive on q_full; early_fetch=True has the
         # MMA warp read the next tile at the start of the current one.
         self.tiles, self.rng, self.q_full_both = list(tiles), rng, q_full_both
         self.early_fetch = early_fetch
+        self.slots = slots
         B = Barrier
         # Barriers of each CTA (index 0 = leader, 1 = peer), as the kernel initialises them.
         self.bar = []
@@ -103,7 +104,7 @@ class Model:
                 d[f"p_full{i}"] = B(f"p_full{i}@{r}", 8)
                 d[f"o_full{i}"] = B(f"o_full{i}@{r}", 1)
                 d[f"o_empty{i}"] = B(f"o_empty{i}@{r}", 8)
-            for s in range(SLOTS):
+            for s in range(self.slots):
                 d[f"full_kv{s}"] = B(f"full_kv{s}@{r}", 1)
                 d[f"empty_k{s}"] = B(f"empty_k{s}@{r}", 1)
                 d[f"empty_v{s}"] = B(f"empty_v{s}@{r}", 1)
@@ -115,8 +116,8 @@ class Model:
         # Buffer contents (tags), per CTA.
         self.ring = [[("init",)] * TILE_SLOTS for _ in range(2)]
         self.q = [[None, None] for _ in range(2)]
-        self.kbuf = [[None] * SLOTS for _ in range(2)]
-        self.vbuf = [[None] * SLOTS for _ in range(2)]
+        self.kbuf = [[None] * self.slots for _ in range(2)]
+        self.vbuf = [[None] * self.slots for _ in range(2)]
         # TMEM of each CTA, per sub-tile: S_i (P_i overwrites half of it) and
         # O_i, with how many of the group's 4 warps have read S / written P /
         # read O (each warp owns 32 of the 128 rows).
@@ -193,12 +194,12 @@ class Model:
                 elif leader or self.q_full_both:
                     qf.arrive()
             for n in range(max(nb)):
-                slot = blk % SLOTS
-                yield Wait(bme[f"empty_k{slot}"], blk // SLOTS - 1, f"producer@{r} empty_k")
+                slot = blk % self.slots
+                yield Wait(bme[f"empty_k{slot}"], blk // self.slots - 1, f"producer@{r} empty_k")
                 if leader:
                     bl[f"full_kv{slot}"].arrive(expect_tx=2 * KV_BYTES)
                 self.tma(r, self.kbuf, slot, ("k", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
-                yield Wait(bme[f"empty_v{slot}"], blk // SLOTS - 1, f"producer@{r} empty_v")
+                yield Wait(bme[f"empty_v{slot}"], blk // self.slots - 1, f"producer@{r} empty_v")
                 self.tma(r, self.vbuf, slot, ("v", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
                 blk += 1
             k += 1
@@ -215,7 +216,7 @@ class Model:
         def issue_s(i, b, k, n):
             def op():
                 expect([self.q[r][i] for r in (0, 1)], ("q", k, i), f"S{i} reads Q")
-                expect([self.kbuf[r][b % SLOTS] for r in (0, 1)], ("k", b), f"S{i} reads K")
+                expect([self.kbuf[r][b % self.slots] for r in (0, 1)], ("k", b), f"S{i} reads K")
                 for r in (0, 1):
                     if self.s[r][i] is not None and self.s_reads[r][i] < 4:
                         raise ProtocolError(f"S{i}({k},{n}) overwrites S {self.s[r][i]} before "
@@ -228,7 +229,7 @@ class Model:
 
         def issue_pv(i, b, k, n):
             def op():
-                expect([self.vbuf[r][b % SLOTS] for r in (0, 1)], ("v", b), f"PV{i} reads V")
+                expect([self.vbuf[r][b % self.slots] for r in (0, 1)], ("v", b), f"PV{i} reads V")
                 for r in (0, 1):
                     if self.p[r][i] != ("p", k, n) or self.p_writes[r][i] != 4:
                         raise ProtocolError(f"PV{i}({k},{n}) reads P {self.p[r][i]} written by "
@@ -256,13 +257,13 @@ class Model:
             for i in (0, 1):
                 yield Wait(bl[f"q_full{i}"], k, f"mma q_full{i}")
             if max(n) > 0:
-                yield Wait(bl[f"full_kv{b % SLOTS}"], b // SLOTS, "mma full_kv")
+                yield Wait(bl[f"full_kv{b % self.slots}"], b // self.slots, "mma full_kv")
                 for i in (0, 1):
                     if n[i] > 0:
                         issue_s(i, b, k, 0)
                     if n[i] <= 1:
                         self.commit([f"q_empty{i}"], 0x3)
-                self.commit([f"empty_k{b % SLOTS}"], 0x3)
+                self.commit([f"empty_k{b % self.slots}"], 0x3)
             else:
                 for i in (0, 1):
                     self.commit([f"q_empty{i}"], 0x3)
@@ -286,7 +287,7 @@ class Model:
                 next_s = [nbn[0] > 0, nbn[1] > 0] if last else [n + 1 < nb[0], n + 1 < nb[1]]
                 more = next_s[0] or next_s[1]
                 if more:
-                    yield Wait(bl[f"full_kv{(b + 1) % SLOTS}"], (b + 1) // SLOTS, "mma full_kv")
+                    yield Wait(bl[f"full_kv{(b + 1) % self.slots}"], (b + 1) // self.slots, "mma full_kv")
                 for i in (0, 1):
                     if n < nb[i]:
                         if n == 0:
@@ -298,7 +299,7 @@ class Model:
                             self.commit([f"o_full{i}"], 0x3)
                             o_cnt[i] += 1
                     if i == 1:
-                        self.commit([f"empty_v{b % SLOTS}"], 0x3)
+                        self.commit([f"empty_v{b % self.slots}"], 0x3)
                     if last and nxt is not INVALID:
                         yield Wait(bl[f"q_full{i}"], k + 1, f"mma q_full{i}")
                     if next_s[i]:
@@ -310,7 +311,7 @@ class Model:
                     elif last and nxt is not INVALID:
                         self.commit([f"q_empty{i}"], 0x3)
                 if more:
-                    self.commit([f"empty_k{(b + 1) % SLOTS}"], 0x3)
+                    self.commit([f"empty_k{(b + 1) % self.slots}"], 0x3)
             if nblk == 0 and nxt is not INVALID:
                 yield from start_tile(nxt, blk, k + 1)
             blk += nblk

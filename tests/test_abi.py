@@ -229,3 +229,11 @@ def _call_split(**over):
                                   dict(out=8), dict(causal=2)])
 def test_splitkv_call_rejects_bad_arguments(over):
     assert _call_split(**over) == _lib.MLA_ERR_INVALID_ARG
+
+
+def test_dims_call_rejects_unsupported_geometries():
+    P = ctypes.c_void_p
+    f = mla.load().mla_prefill_fwd_dims
+    for qk, v in ((64, 128), (192, 64), (320, 128), (192, 512)):
+        assert f(P(16), P(16), P(16), P(16), P(16), 4, 4, 0.1, 1, P(16), None, None, 1, 1, 4, 4,
+                 qk, v, P(64), 4096) == _lib.MLA_ERR_INVALID_ARG

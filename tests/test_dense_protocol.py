@@ -62,3 +62,12 @@ def test_model_catches_an_early_next_tile_read():
     slots those loads wait for the MMA warp."""
     with pytest.raises(dp.ProtocolError, match="deadlock"):
         dp.run_case([(5, 6), (1, 1)], 0, early_fetch=True)
+
+
+def test_protocol_holds_with_two_kv_slots():
+    """The 256-wide qk geometry keeps two K/V slots instead of three."""
+    rng = random.Random(11)
+    for seed in range(150):
+        tiles = [(rng.choice([0, 1, 2, 3, 5]), rng.choice([0, 1, 2, 4, 6]))
+                 for _ in range(rng.randint(1, 8))]
+        dp.run_case(tiles, seed, slots=2)

@@ -427,3 +427,38 @@ def test_splitkv_is_deterministic_and_close_to_unsplit():
     o_p, l_p = run_dense(case)
     assert (a.float() - o_p.float()).abs().max().item() <= 2 ** -7
     assert (la - l_p).abs().max().item() <= 1e-4
+
+
+# ------------------------------------------------------ other MLA head geometries
+@pytest.mark.parametrize("qk,v", [(256, 256), (128, 128), (256, 128), (128, 256)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_other_head_geometries(qk, v, causal):
+    """vLLM's supports_mla_dimensions rows (192+64, 256), (64+64, 128),
+    (256+0, 256), and the mixed widths, on a ragged batch with tile edges
+    and rows without keys."""
+    import mla_prefill_attention_causal_b200 as mla
+    lens_q = [300, 129, 1, 513]
+    lens_k = [300, 129, 1, 513] if causal else [256, 40, 7, 600]
+    case = syn.dense_case(lens_q, lens_k, 3, seed=qk + v + causal, causal=causal, qk_dim=qk,
+                          v_dim=v)
+    out, lse = mla.mla_prefill_fwd_dims(dev_bf16(case["q"]), dev_bf16(case["k"]),
+                                        dev_bf16(case["v"]), dev_i32(case["cu_q"]),
+                                        dev_i32(case["cu_k"]), case["max_q"], case["max_k"],
+                                        case["scale"], causal=causal)
+    torch.cuda.synchronize()
+    assert out.shape == (sum(lens_q), 3, v)
+    ref_o, ref_l = oracle.dense_prefill(case["q"], case["k"], case["v"], case["cu_q"],
+                                        case["cu_k"], case["scale"], causal)
+    assert_out_close(to_f64(out), ref_o, f"qk {qk} v {v} out")
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), ref_l, f"qk {qk} v {v} lse")
+
+
+def test_dims_call_with_the_default_geometry_is_the_plain_call():
+    import mla_prefill_attention_causal_b200 as mla
+    case = syn.dense_case([700, 129], [700, 129], 4, seed=104)
+    out, lse = mla.mla_prefill_fwd_dims(dev_bf16(case["q"]), dev_bf16(case["k"]),
+                                        dev_bf16(case["v"]), dev_i32(case["cu_q"]),
+                                        dev_i32(case["cu_k"]), case["max_q"], case["max_k"],
+                                        case["scale"], causal=True)
+    o_p, l_p = run_dense(case)
+    assert torch.equal(out, o_p) and torch.equal(lse, l_p)

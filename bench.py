@@ -195,6 +195,8 @@ class DenseWorkload:
     kernel = "mla::dense::dense_fwd_kernel"
     sources = ("dense_fwd.cuh", "ptx.cuh")
     profile = "dense_fwd_varlen16k.md"
+    in_attrs = ("q", "k", "v", "cu")  # device inputs, in the order of self.hin
+    out_attrs = ("out", "lse")        # device outputs, in the order of self.hout
 
     def __init__(self, dev, seed, heads, long=False):
         import torch
@@ -221,13 +223,6 @@ class DenseWorkload:
         c = self.case
         mla.mla_prefill_fwd(self.q, self.k, self.v, self.cu, self.cu, c["max_q"], c["max_q"],
                             c["scale"], causal=True, out=self.out, lse=self.lse)
-
-    def e2e_step(self):
-        for d, h in zip((self.q, self.k, self.v, self.cu), self.hin):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.hout[0].copy_(self.out, non_blocking=True)
-        self.hout[1].copy_(self.lse, non_blocking=True)
 
     def config(self):
         c = self.case
@@ -304,6 +299,8 @@ class SparseWorkload:
     kernel = "mla::sparse::sparse_fwd_kernel"
     sources = ("sparse_fwd.cuh", "ptx.cuh")
     profile = "sparse_fwd_4k.md"
+    in_attrs = ("q", "kv", "idx")
+    out_attrs = ("out", "lse")
     data = "synthetic (seeded N(0,1) bf16 q and latent cache, causal top-k index lists)"
     reference_sample = "step i = all 128 heads of token (i * 997 mod 4096)"
 
@@ -331,13 +328,6 @@ class SparseWorkload:
         import mla_prefill_attention_causal_b200 as mla
         mla.mla_sparse_prefill_fwd(self.q, self.kv, self.idx, self.case["scale"], out=self.out,
                                    lse=self.lse)
-
-    def e2e_step(self):
-        for d, h in zip((self.q, self.kv, self.idx), self.hin):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.hout[0].copy_(self.out, non_blocking=True)
-        self.hout[1].copy_(self.lse, non_blocking=True)
 
     def config(self):
         c = self.case
@@ -384,6 +374,8 @@ class ChunkedWorkload:
     profile = "dense_fwd_chunked.md"  # DRAM bytes of the step's two attention launches
     merge_sources = ("merge.cuh",)
     merge_profile = "merge_chunked.md"
+    in_attrs = ("q", "kp", "vp", "ks", "vs", "cu_q", "cu_p")
+    out_attrs = ("out", "lse")
     data = "synthetic (seeded N(0,1) bf16 query chunks, prefix and self K/V)"
     reference_sample = ("step i = head (i mod 128) of sequence (i mod 4): prefix pass, self pass "
                         "and merge of that head's 2048 query rows")
@@ -430,14 +422,6 @@ class ChunkedWorkload:
             self.merge_events.append((e0, e1))
         else:
             mla.mla_attn_merge(self.op, self.lp, self.os, self.ls, out=self.out, lse_out=self.lse)
-
-    def e2e_step(self):
-        for d, h in zip((self.q, self.kp, self.vp, self.ks, self.vs, self.cu_q, self.cu_p),
-                        self.hin):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.hout[0].copy_(self.out, non_blocking=True)
-        self.hout[1].copy_(self.lse, non_blocking=True)
 
     def config(self):
         c = self.case
@@ -517,6 +501,7 @@ class SplitKvWorkload(DenseWorkload):
     metric = ("MLA prefill attn TFLOPS (causal-adj), split-KV on a few-tile shape, "
               "% of B200 dense BF16 peak, 1 GPU")
     profile = "dense_fwd_splitkv.md"
+    in_attrs = ("q", "k", "v", "cu", "cuk")
 
     def __init__(self, dev, seed, heads):
         import torch
@@ -554,13 +539,6 @@ class SplitKvWorkload(DenseWorkload):
 
     def step(self):
         self._call(self.splits, self.ws)
-
-    def e2e_step(self):
-        for d, h in zip((self.q, self.k, self.v, self.cu, self.cuk), self.hin):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.hout[0].copy_(self.out, non_blocking=True)
-        self.hout[1].copy_(self.lse, non_blocking=True)
 
     def time_unsplit(self, steps):
         import torch
@@ -604,6 +582,60 @@ class SplitKvWorkload(DenseWorkload):
         return oracle.dense_flops(c["lens_q"], c["lens_k"], 1, True), time.perf_counter() - t0
 
     reference_sample = "step i = head (i mod 16) of the whole call"
+
+
+def time_e2e(w, steps: int) -> float:
+    """Milliseconds per step of the end-to-end run: every step copies its
+    inputs from pinned host memory, runs the call and reads its outputs back
+    to pinned host memory.  Two device buffer sets alternate between steps,
+    so step i+1's host-to-device copy (its own stream) overlaps step i's
+    kernels and device-to-host copy (two more streams); events order each
+    set's reuse.  Timed from before the first copy to after the last one."""
+    import torch
+    sets = [{a: getattr(w, a) for a in w.in_attrs + w.out_attrs}]
+    sets.append({a: torch.empty_like(t) for a, t in sets[0].items()})
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    h2d_done = [torch.cuda.Event(), torch.cuda.Event()]
+    run_done = [torch.cuda.Event(), torch.cuda.Event()]
+    d2h_done = [torch.cuda.Event(), torch.cuda.Event()]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def one(i):
+        b = i % 2
+        buf = sets[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(run_done[b])       # step i-2's kernels are done with the inputs
+            for a, h in zip(w.in_attrs, w.hin):
+                buf[a].copy_(h, non_blocking=True)
+            h2d_done[b].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(h2d_done[b])
+            if i >= 2:
+                s_run.wait_event(d2h_done[b])      # step i-2's outputs have been read back
+            for a, t in buf.items():
+                setattr(w, a, t)
+            w.step()
+            run_done[b].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(run_done[b])
+            for a, h in zip(w.out_attrs, w.hout):
+                h.copy_(buf[a], non_blocking=True)
+            d2h_done[b].record(s_out)
+
+    one(0)
+    one(1)
+    torch.cuda.synchronize()
+    t0.record(s_in)
+    for i in range(steps):
+        one(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_run)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    for a, t in sets[0].items():
+        setattr(w, a, t)
+    return t0.elapsed_time(t1) / steps
 
 
 def rank_seed(base: int, rank: int, world: int) -> int:
@@ -747,16 +779,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     # End to end through the public call with host buffers: H2D of the step's
     # inputs from pinned memory, the kernel(s), D2H of out and lse.
     e2e_steps = max(3, min(args.steps, 20))
-    w.e2e_step()
-    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        w.e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, world, dev)
+    e2e_ms = max_over_ranks(time_e2e(w, e2e_steps), world, dev)
     h2d = sum(x.numel() * x.element_size() for x in w.hin)
     d2h = sum(x.numel() * x.element_size() for x in w.hout)
 
@@ -782,7 +807,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                      "kernel": w.kernel,
                      "timed": "one public call per step; CUDA events on its stream"},
         "e2e": {"value": whole_job_value(w.flops, world, e2e_ms), "unit": UNIT,
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipelined": "two device buffer sets: a step's host-to-device copy overlaps the "
+                             "previous step's kernels and device-to-host copy"},
         "gpu_launches": args.steps * w.launches,
         "clocks": clocks,
         "device_status": status,

@@ -33,7 +33,8 @@ the sum of all ranks' FLOPs over the slowest rank's time.
 
 Timing: CUDA events on the launching stream; the inputs (Q+K+V = 2.08 GB for
 the dense workload) are larger than the 126 MB L2, so nothing is flushed
-between steps.  The roofline fraction is given against the measured burst
+between steps; the splitkv workload's inputs fit in L2, so a 256 MB buffer is
+written before each of its calls and each call is timed alone.  The roofline fraction is given against the measured burst
 bf16 peak and, as ``frac_of_sustained``, against the measured sustained one;
 the default 30 timed calls match the burst measurement, while a few hundred
 back-to-back calls run under the power cap and land near the sustained
@@ -63,6 +64,7 @@ WORKLOAD = ("dense varlen causal MLA prefill: 8 sequences, lengths U[512,4096] (
             "fp32 LSE")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
+L2_FLUSH_BYTES = 256 << 20  # written between timed calls of workloads smaller than the 126 MB L2
 
 
 def load_peaks():
@@ -502,6 +504,7 @@ class SplitKvWorkload(DenseWorkload):
               "% of B200 dense BF16 peak, 1 GPU")
     profile = "dense_fwd_splitkv.md"
     in_attrs = ("q", "k", "v", "cu", "cuk")
+    flush_l2 = True
 
     def __init__(self, dev, seed, heads):
         import torch
@@ -540,17 +543,20 @@ class SplitKvWorkload(DenseWorkload):
     def step(self):
         self._call(self.splits, self.ws)
 
-    def time_unsplit(self, steps):
+    def time_unsplit(self, steps, flush):
         import torch
         for _ in range(3):
             self._call(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        ms = 0.0
         for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
             self._call(1)
-        e1.record()
-        torch.cuda.synchronize()
-        self.unsplit_ms = e0.elapsed_time(e1) / steps
+            e1.record()
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
+        self.unsplit_ms = ms / steps
 
     def config(self):
         c = self.case
@@ -559,8 +565,10 @@ class SplitKvWorkload(DenseWorkload):
                              "1/sqrt(192)" % self.H),
                 "heads": self.H, "num_splits": self.splits, "flops_per_step": self.flops,
                 "unsplit_ms": self.unsplit_ms,
-                "l2": "inputs %.1f MB < L2: repeated calls read K/V from L2 (a launch-bound "
-                      "shape)" % ((self.q.numel() + self.k.numel() + self.v.numel()) * 2 / 1e6)}
+                "l2": ("inputs %.1f MB < L2: a %d MB buffer is written before every timed "
+                       "call, each call timed alone with CUDA events"
+                       % ((self.q.numel() + self.k.numel() + self.v.numel()) * 2 / 1e6,
+                          L2_FLUSH_BYTES >> 20))}
 
     data = "synthetic (seeded N(0,1) bf16)"
 
@@ -750,21 +758,36 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if hasattr(w, "merge_events"):
         w.merge_events = []
+    flush = (torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+             if getattr(w, "flush_l2", False) else None)
+    step_events = []
     ev0.record(stream)
     for _ in range(args.steps):
+        if flush is None:
+            w.step()
+            continue
+        # Inputs smaller than L2: write a buffer larger than L2 before every
+        # call and time the call alone.
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         w.step()
+        b.record(stream)
+        step_events.append((a, b))
     ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     if hasattr(w, "time_unsplit"):
-        w.time_unsplit(args.steps)  # outside the timed region, for comparison
+        w.time_unsplit(args.steps, flush)  # outside the timed region, for comparison
     merge_ms = None
     if getattr(w, "merge_events", None):
         merge_ms = sum(a.elapsed_time(b) for a, b in w.merge_events) / len(w.merge_events)
         w.merge_events = None
-    ms_total = ev0.elapsed_time(ev1)
+    ms_total = (sum(a.elapsed_time(b) for a, b in step_events) if step_events
+                else ev0.elapsed_time(ev1))
+    del flush
     ms_step = max_over_ranks(ms_total, world, dev) / args.steps
     value = whole_job_value(w.flops, world, ms_step)
     status = mla.mla_device_status(reset=True)

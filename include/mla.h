@@ -227,8 +227,9 @@ int mla_prefill_fwd_ex(const void* q, const void* k, const void* v, const int32_
 size_t mla_prefill_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_splits);
 
 /* A number of splits for a call of these sizes on the current device (1 when
- * the call already has a tile for every CTA pair): enough tiles for every
- * pair, at least two 128-key blocks a split, at most MLA_MAX_SPLITS. */
+ * the call already has a tile for every CTA pair): the fewest splits that
+ * minimise (waves of split tiles over the CTA pairs) x (128-key blocks of a
+ * split + 2), with at least two blocks a split and at most MLA_MAX_SPLITS. */
 int mla_prefill_num_splits(int batch, int total_q, int num_heads, int max_seqlen_q,
                            int max_seqlen_k);
 

@@ -618,11 +618,22 @@ int mla_prefill_num_splits(int batch, int total_q, int num_heads, int max_seqlen
   const long long entries = per_seq * batch < by_total ? per_seq * batch : by_total;
   const long long tiles = entries * num_heads;
   if (tiles <= 0 || tiles >= clusters) return 1;
-  long long n = (clusters + tiles - 1) / tiles;               // enough tiles for every cluster
   const long long blocks = (static_cast<long long>(max_seqlen_k) + kBlockKeys - 1) / kBlockKeys;
-  if (n > blocks / 2) n = blocks / 2;                         // at least two KV blocks a split
-  if (n > MLA_MAX_SPLITS) n = MLA_MAX_SPLITS;
-  return n < 1 ? 1 : static_cast<int>(n);
+  long long n_max = blocks / 2;                               // at least two KV blocks a split
+  if (n_max > MLA_MAX_SPLITS) n_max = MLA_MAX_SPLITS;
+  // The fewest splits that minimise the critical path: waves of split tiles
+  // over the clusters times the blocks of one split, plus about two blocks'
+  // worth of per-tile overhead (Q load, partial store).
+  long long best_n = 1, best_cost = -1;
+  for (long long n = 1; n <= n_max; ++n) {
+    const long long waves = (tiles * n + clusters - 1) / clusters;
+    const long long cost = waves * ((blocks + n - 1) / n + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_n = n;
+    }
+  }
+  return static_cast<int>(best_n);
 }
 
 int mla_prefill_fwd_splitkv(const void* q, const void* k, const void* v,

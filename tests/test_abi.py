@@ -207,7 +207,8 @@ def test_splitkv_sizes_and_choice():
     assert f(2, 100, 8, 3) == parts + 3 * 100 * 8 * 129 * 4
     assert f(2, 100, 8, 0) == 0 and f(2, 100, 8, 65) == 0 and f(2, 100, 0, 2) == 0
     # no GPU here: the choice assumes 74 CTA pairs
-    assert mla.num_splits_for(1, 1, 16, 1, 8192) == 5     # 16 tiles -> ceil(74/16)
+    assert mla.num_splits_for(1, 1, 16, 1, 8192) == 4     # 64 split tiles: one wave on 74 pairs
+    assert mla.num_splits_for(1, 1, 2, 1, 8192) == 32     # 2 x 32 tiles of 2 blocks
     assert mla.num_splits_for(1, 1, 128, 1, 8192) == 1    # a tile for every pair already
     assert mla.num_splits_for(1, 1, 4, 1, 512) == 2       # at least two KV blocks a split
     assert mla.num_splits_for(1, 1, 1, 1, 1 << 20) == 64  # at most MLA_MAX_SPLITS

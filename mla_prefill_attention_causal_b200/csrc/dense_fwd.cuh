@@ -15,7 +15,9 @@
 // halves each SM's K/V traffic and the shared-memory operand bytes per MMA.
 //
 // Work unit ("tile"): (sequence, 512-row query block, head) = two M=256
-// sub-tiles that share every K/V block.  A planner kernel sorts the
+// sub-tiles that share every K/V block.  The query blocks are aligned to the
+// end of the sequence, so that a ragged first block holds the rows that see
+// the fewest keys.  A planner kernel sorts the
 // (sequence, query block) entries by their number of visible KV blocks,
 // longest first, into the caller's workspace.  Tile t of the resulting list
 // is taken head-major (all entries of head 0, then of head 1, ...), except
@@ -174,10 +176,19 @@ struct Params {
 constexpr uint32_t kIdescQK = idesc_bf16_f32(256, 128, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(256, 128, true);
 
+// First row of a sequence's 512-row entry mb.  Entries are aligned to the
+// end of the sequence (entry 0 holds its last 512 rows), so a ragged piece
+// (Lq mod 512 rows) comes first, where rows see the fewest keys; its rows
+// below 0 (and, in every entry, rows past Lq) are computed as masked filler
+// and never stored.  With start-aligned entries the ragged piece would hold
+// the last rows, whose sub-tile walks every KV block for a few rows.
+__host__ __device__ __forceinline__ int entry_row0(int Lq, int mb) {
+  return Lq - (mb + 1) * kTileRows;
+}
 // Number of keys (a prefix [0, n)) that any row of the 256-row sub-tile
 // starting at row0 may see.
 __host__ __device__ __forceinline__ int sub_tile_keys(int row0, int Lq, int Lk, int causal) {
-  if (row0 >= Lq) return 0;
+  if (row0 >= Lq || row0 + kSubRows <= 0) return 0;
   if (!causal) return Lk;
   const int last = min(row0 + kSubRows - 1, Lq - 1);
   return max(0, min(Lk, last + (Lk - Lq) + 1));
@@ -190,7 +201,7 @@ __host__ __device__ __forceinline__ int blocks_for(int keys) {
 // of its own visible keys; none when it has no rows.
 __host__ __device__ __forceinline__ int sub_tile_blocks(int row0, int Lq, int Lk, int Lc,
                                                         int causal) {
-  if (row0 >= Lq) return 0;
+  if (row0 >= Lq || row0 + kSubRows <= 0) return 0;
   return blocks_for(Lc) + blocks_for(sub_tile_keys(row0, Lq, Lk, causal));
 }
 // Split-KV: a tile's block sequence (nmax = the longer sub-tile's blocks) is
@@ -218,7 +229,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   if (tid == 0) s_total = 0;
   __syncthreads();
   auto work_of = [&](int Lq, int Lk, int Lc, int mb) -> int {
-    const int m0 = mb * kTileRows;
+    const int m0 = entry_row0(Lq, mb);
     const int n0 = sub_tile_blocks(m0, Lq, Lk, Lc, causal);
     const int n1 = sub_tile_blocks(m0 + kSubRows, Lq, Lk, Lc, causal);
     return min(kPlanBins - 1, max(n0, n1));
@@ -327,7 +338,7 @@ __device__ __forceinline__ TileInfo tile_info(const Params& p, int t, int num_ti
     ti.Lk = p.cu_k[en.x + 1] - ti.k_start;
     ti.c_start = p.cu_ctx != nullptr ? p.cu_ctx[en.x] : 0;
     ti.Lc = p.cu_ctx != nullptr ? p.cu_ctx[en.x + 1] - ti.c_start : 0;
-    ti.m0 = en.y * kTileRows;
+    ti.m0 = entry_row0(ti.Lq, en.y);
     ti.hs = h | (split << 16);
   } else {
     ti.q_start = ti.Lq = ti.k_start = ti.Lk = ti.c_start = ti.Lc = ti.m0 = ti.hs = 0;
@@ -833,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // is O_acc / l and m + log2 l.  A row that saw no key keeps m_run =
       // -inf (its weights are only the tiny clamped values of the polynomial
       // path): output 0, LSE -inf, or the sink's logit.
-      const bool row_ok = r < e_lq;
+      const bool row_ok = r >= 0 && r < e_lq;
       const size_t row_index = static_cast<size_t>(e_q0 + r) * p.num_heads + e_h;
       const size_t out_off = static_cast<size_t>(e_q0 + r) * p.out_rs +
                              static_cast<size_t>(e_h) * p.out_hs;  // first element of the row

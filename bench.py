@@ -425,6 +425,25 @@ class ChunkedWorkload:
         else:
             mla.mla_attn_merge(self.op, self.lp, self.os, self.ls, out=self.out, lse_out=self.lse)
 
+    def time_merge_alone(self, steps, flush_bytes):
+        """Milliseconds of one merge launch alone: after a write of a buffer
+        larger than L2 (so that neither its inputs nor the attention
+        passes' unwritten outputs sit in L2), CUDA events around the merge."""
+        import torch
+        import mla_prefill_attention_causal_b200 as mla
+        flush = torch.empty(flush_bytes, dtype=torch.uint8, device=self.out.device)
+        ms = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mla.mla_attn_merge(self.op, self.lp, self.os, self.ls, out=self.out, lse_out=self.lse)
+            e1.record()
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
+        return ms / steps
+
     def config(self):
         c = self.case
         return {"workload": ("chunked MLA prefill with context: %d sequences, %d-token query "
@@ -847,7 +866,15 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                                   "peak_source": f"{peak_src} hbm_gbs",
                                   "traffic": recorded_traffic_for(w.merge_profile,
                                                                   w.merge_sources),
-                                  "kernel": "mla::merge::merge_kernel"}
+                                  "kernel": "mla::merge::merge_kernel",
+                                  "timed": ("inside the step, right after the two attention "
+                                            "passes (whose outputs are still being written "
+                                            "back from L2)")}
+        alone_ms = w.time_merge_alone(10, L2_FLUSH_BYTES)
+        alone_gbs = w.merge_bytes / (alone_ms * 1e-3) / 1e9
+        line["merge_roofline"]["alone"] = {"ms": alone_ms, "achieved": alone_gbs,
+                                           "frac": alone_gbs / hbm,
+                                           "timed": "10 launches, each after an L2 flush"}
     if world == 1 and not args.no_cpu_baseline:
         f, dt, sample = w.oracle_sample()
         line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": UNIT, "cores": blas_threads(),

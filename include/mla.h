@@ -271,8 +271,8 @@ int mla_prefill_fwd_dims(const void* q, const void* k, const void* v,
  * (The pages have no counterpart to this entry point; it is a convenience of
  * this library.)  Some callers have no way to obtain the workspace that
  * mla_prefill_fwd needs: code that must not call cudaMalloc at all (for
- * example while other work is being recorded, or inside a runtime that owns
- * every allocation), or a plain C caller with no allocator of its own.  This
+ * example inside a runtime that owns every device allocation and hands out
+ * none), or a plain C caller with no allocator of its own.  This
  * variant takes the same arguments minus the workspace and runs the same
  * kernels with their work list in a fixed scratch array that is part of the
  * library itself (MLA_NOALLOC_SCRATCH_BYTES of device memory, reserved on
@@ -285,8 +285,7 @@ int mla_prefill_fwd_dims(const void* q, const void* k, const void* v,
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and keeps it for
  *     that device's CUDA context; a context created anew (for example
- *     after cudaDeviceReset) gets the lookup again on its first call.  Make
- *     that first call before capturing work into a graph on that device.
+ *     after cudaDeviceReset) gets the lookup again on its first call.
  *   - All calls share the one array.  The kernels rewrite everything they
  *     read from it, so nothing needs clearing between calls, but two calls
  *     whose kernels can overlap on the GPU (different streams without an

@@ -234,24 +234,23 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ER
 // cached here.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
 struct NoallocScratch {
-  std::atomic<unsigned long long> ctx{0};  // context `ptr` belongs to (0: none)
-  std::atomic<void*> ptr{nullptr};
+  unsigned long long ctx = 0;  // context `ptr` belongs to (0: none)
+  void* ptr = nullptr;
 };
-NoallocScratch g_noalloc[kMaxDevices];
+NoallocScratch g_noalloc[kMaxDevices];  // guarded by g_noalloc_mu
 std::mutex g_noalloc_mu;
 
 // Device address of the scratch array in the current context of `dev`
-// (prepare_device has made that context current).
+// (prepare_device has made that context current).  The cache is read and
+// written under one mutex, so the context id and the address always belong
+// together, also when several contexts of a device are used from different
+// threads; a context id of 0 (not known) is never cached.
 int noalloc_scratch(int dev, void** out) {
-  NoallocScratch& n = g_noalloc[dev];
   const unsigned long long ctx = current_context_id();
-  if (ctx != 0 && n.ctx.load(std::memory_order_acquire) == ctx) {
-    *out = n.ptr.load(std::memory_order_relaxed);
-    return MLA_OK;
-  }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (ctx != 0 && n.ctx.load(std::memory_order_relaxed) == ctx) {
-    *out = n.ptr.load(std::memory_order_relaxed);
+  NoallocScratch& n = g_noalloc[dev];
+  if (ctx != 0 && n.ctx == ctx) {
+    *out = n.ptr;
     return MLA_OK;
   }
   void* p = nullptr;
@@ -259,8 +258,8 @@ int noalloc_scratch(int dev, void** out) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }
-  n.ptr.store(p, std::memory_order_relaxed);
-  n.ctx.store(ctx, std::memory_order_release);
+  n.ptr = p;
+  n.ctx = ctx;
   *out = p;
   return MLA_OK;
 }

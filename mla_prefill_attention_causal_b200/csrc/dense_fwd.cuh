@@ -498,6 +498,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_blocks(ti, causal, p.nsplit, nb, lo);
         const int h = ti.head();
         const int nblk = max(nb[0], nb[1]);
+        // The tile's first K/V block goes out before its Q: its ring slot is
+        // freed by MMAs three blocks back, while Q's buffers wait for the
+        // previous tile's last S MMAs -- so the MMA warp, which needs block 0
+        // at the previous tile's last block, does not wait for the Q reload.
+        const int nctx = blocks_for(ti.Lc);  // the context's blocks come first
+        auto issue_kv = [&](int n) -> bool {  // block n of the tile, the blk-th overall
+          const int slot = blk % kSlots;
+          const uint32_t par = (static_cast<uint32_t>(blk / kSlots) & 1u) ^ 1u;
+          const int bi = lo + n;  // block of the tile's sequence
+          const bool in_ctx = bi < nctx;
+          const int key0 = in_ctx ? ti.c_start + bi * kBlockKeys
+                                  : ti.k_start + (bi - nctx) * kBlockKeys;
+          const CUtensorMap* mk = in_ctx ? &tm_kc : &tm_k;
+          const CUtensorMap* mv = in_ctx ? &tm_vc : &tm_v;
+          // K: this CTA's 64 keys, three 64-dim chunks of the 192
+          if (!wait(smem_u32(&bars->empty_k[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD))
+            return false;
+          // one barrier per block for K and V: the MMA warp waits once per block
+          if (leader)
+            mbar_arrive_expect_tx(smem_u32(&bars->full_kv[slot]), 2 * (kKSlotBytes + kVSlotBytes));
+          const uint32_t kbar = lead(&bars->full_kv[slot]);
+#pragma unroll
+          for (int u = 0; u < kKUnits; ++u)
+            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, mk, 64 * u, h,
+                             key0 + static_cast<int>(rank) * kHalfKeys, kbar, pol_kv);
+          ++blk;  // issued (its V follows on the same barrier)
+          // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
+          if (!wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD))
+            return false;
+#pragma unroll
+          for (int u = 0; u < kVUnits; ++u)
+            tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, mv,
+                             static_cast<int>(rank) * kHalfDv, h, key0 + 64 * u, kbar, pol_kv);
+          return true;
+        };
+        if (nblk > 0) ok = issue_kv(0);
         // Q rows of this CTA, once the previous tile's last S MMA has read them.
         for (int i = 0; i < 2 && ok; ++i) {
           if (!(ok = wait(smem_u32(&bars->q_empty[i]), (static_cast<uint32_t>(k) & 1u) ^ 1u,
@@ -524,36 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_cluster(qbar);
           }
         }
-        const int nctx = blocks_for(ti.Lc);  // the context's blocks come first
-        for (int n = 0; n < nblk && ok; ++n, ++blk) {
-          const int slot = blk % kSlots;
-          const uint32_t par = (static_cast<uint32_t>(blk / kSlots) & 1u) ^ 1u;
-          const int bi = lo + n;  // block of the tile's sequence
-          const bool in_ctx = bi < nctx;
-          const int key0 = in_ctx ? ti.c_start + bi * kBlockKeys
-                                  : ti.k_start + (bi - nctx) * kBlockKeys;
-          const CUtensorMap* mk = in_ctx ? &tm_kc : &tm_k;
-          const CUtensorMap* mv = in_ctx ? &tm_vc : &tm_v;
-          // K: this CTA's 64 keys, three 64-dim chunks of the 192
-          if (!(ok = wait(smem_u32(&bars->empty_k[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
-            break;
-          // one barrier per block for K and V: the MMA warp waits once per block
-          if (leader)
-            mbar_arrive_expect_tx(smem_u32(&bars->full_kv[slot]), 2 * (kKSlotBytes + kVSlotBytes));
-          const uint32_t kbar = lead(&bars->full_kv[slot]);
-#pragma unroll
-          for (int u = 0; u < kKUnits; ++u)
-            tma_load_3d_pair(sRingK + slot * kKSlotBytes + u * kUnitBytes, mk, 64 * u, h,
-                             key0 + static_cast<int>(rank) * kHalfKeys, kbar, pol_kv);
-          // V: all 128 keys (two units of 64), this CTA's 64 of the 128 value dims
-          if (!(ok = wait(smem_u32(&bars->empty_v[slot]), par, MLA_DEVSTAT_WAIT_TIMEOUT_LOAD)))
-            break;
-          const uint32_t vbar = kbar;
-#pragma unroll
-          for (int u = 0; u < kVUnits; ++u)
-            tma_load_3d_pair(sRingV + slot * kVSlotBytes + u * kUnitBytes, mv,
-                             static_cast<int>(rank) * kHalfDv, h, key0 + 64 * u, vbar, pol_kv);
-        }
+        for (int n = 1; n < nblk && ok; ++n) ok = issue_kv(n);
       }
       if (!ok && leader) {
         // Unwinding: let the copies already issued land before the CTA exits.

@@ -182,6 +182,19 @@ class Model:
             if ti is INVALID:
                 return
             nb = (sub_blocks(ti, 0), sub_blocks(ti, 1))
+
+            def load_kv(blk):
+                slot = blk % self.slots
+                yield Wait(bme[f"empty_k{slot}"], blk // self.slots - 1, f"producer@{r} empty_k")
+                if leader:
+                    bl[f"full_kv{slot}"].arrive(expect_tx=2 * KV_BYTES)
+                self.tma(r, self.kbuf, slot, ("k", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
+                yield Wait(bme[f"empty_v{slot}"], blk // self.slots - 1, f"producer@{r} empty_v")
+                self.tma(r, self.vbuf, slot, ("v", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
+
+            # the tile's first K/V block goes out before its Q
+            if max(nb) > 0:
+                yield from load_kv(blk)
             for i in (0, 1):
                 yield Wait(bme[f"q_empty{i}"], k - 1, f"producer@{r} q_empty{i} tile {k}")
                 qf = bl[f"q_full{i}"]
@@ -193,15 +206,9 @@ class Model:
                     self.tma(r, self.q, i, ("q", k, i), qf, Q_BYTES)
                 elif leader or self.q_full_both:
                     qf.arrive()
-            for n in range(max(nb)):
-                slot = blk % self.slots
-                yield Wait(bme[f"empty_k{slot}"], blk // self.slots - 1, f"producer@{r} empty_k")
-                if leader:
-                    bl[f"full_kv{slot}"].arrive(expect_tx=2 * KV_BYTES)
-                self.tma(r, self.kbuf, slot, ("k", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
-                yield Wait(bme[f"empty_v{slot}"], blk // self.slots - 1, f"producer@{r} empty_v")
-                self.tma(r, self.vbuf, slot, ("v", blk), bl[f"full_kv{slot}"], KV_BYTES // 2)
-                blk += 1
+            for n in range(1, max(nb)):
+                yield from load_kv(blk + n)
+            blk += max(nb)
             k += 1
 
     def mma_warp(self):

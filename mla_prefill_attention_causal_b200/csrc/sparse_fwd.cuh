@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
         }
         ok = __all_sync(0xffffffffu, ok);
-        __nanosleep(32);
+        __nanosleep(8);
       }
     }
     tc_commit_elect(smem_u32(&bars->o_full));
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          if ((j & 7) < 5)
+          if ((j & 7) < 7)  // 14 of every 16 pairs on the MUFU unit, 2 on the FMA pipe
             pk[j] = softmax_pair_mufu(x[32 * cc + 2 * j], x[32 * cc + 2 * j + 1], c2, negm2,
                                       acc[j & 3]);
           else

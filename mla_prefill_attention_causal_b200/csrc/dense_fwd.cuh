@@ -163,6 +163,7 @@ struct Params {
   const float* out_scale;  // e4m3 output scale (device scalar), or null: bf16 output
   float* o_part;           // split-KV: fp32 [nsplit][total_q][H][128] partial outputs
   float* lse_part;         // split-KV: fp32 [nsplit][H][total_q] partial LSEs
+  int wide_out;            // bit 0: every out row is 32-byte aligned; bit 1: every o_part row is
   int nsplit;              // KV splits per tile (1: none; the partials are unused)
   WsHeader* ws;
   const int2* entries;  // [E] {sequence, 512-row block index}, longest first
@@ -356,6 +357,15 @@ __device__ __forceinline__ void tile_blocks(const TileInfo& t, int causal, int n
   lo = split_lo(nmax, t.split(), nsplit);
   n[0] = split_count(f0, nmax, t.split(), nsplit);
   n[1] = split_count(f1, nmax, t.split(), nsplit);
+}
+
+// 32-byte store (the address must be 32-byte aligned).  A thread writes one
+// output row; in 32-byte pieces each store fills whole L2 sectors, where
+// 16-byte pieces leave every sector to two separate partial writes.
+__device__ __forceinline__ void st_global_v8(void* addr, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
@@ -884,39 +894,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (row_ok && p.nsplit > 1) {
           // split-KV: this split's O (normalised by its own sum) in fp32
-          float4* prow = reinterpret_cast<float4*>(
-              p.o_part + (static_cast<size_t>(e_split) * p.total_q * p.num_heads + row_index) * kDv);
+          float* prow =
+              p.o_part + (static_cast<size_t>(e_split) * p.total_q * p.num_heads + row_index) * kDv;
+          if (p.wide_out & 2) {
 #pragma unroll
-          for (int v4 = 0; v4 < 32; ++v4)
-            prow[v4] = make_float4(__uint_as_float(o[4 * v4]) * scale_o,
-                                   __uint_as_float(o[4 * v4 + 1]) * scale_o,
-                                   __uint_as_float(o[4 * v4 + 2]) * scale_o,
-                                   __uint_as_float(o[4 * v4 + 3]) * scale_o);
+            for (int v8 = 0; v8 < 16; ++v8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = __float_as_uint(__uint_as_float(o[8 * v8 + j]) * scale_o);
+              st_global_v8(prow + 8 * v8, w);
+            }
+          } else {
+            float4* prow4 = reinterpret_cast<float4*>(prow);
+#pragma unroll
+            for (int v4 = 0; v4 < 32; ++v4)
+              prow4[v4] = make_float4(__uint_as_float(o[4 * v4]) * scale_o,
+                                      __uint_as_float(o[4 * v4 + 1]) * scale_o,
+                                      __uint_as_float(o[4 * v4 + 2]) * scale_o,
+                                      __uint_as_float(o[4 * v4 + 3]) * scale_o);
+          }
         } else if (row_ok && !fp8) {
-          uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + out_off);
+          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + out_off;
+          if (p.wide_out & 1) {
 #pragma unroll
-          for (int v4 = 0; v4 < 16; ++v4) {
-            uint32_t pk[4];
+            for (int v8 = 0; v8 < 8; ++v8) {  // 16 bf16 per store
+              uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * scale_o,
-                                  __uint_as_float(o[8 * v4 + 2 * j + 1]) * scale_o);
-            orow[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              for (int j = 0; j < 8; ++j)
+                pk[j] = pack_bf16x2(__uint_as_float(o[16 * v8 + 2 * j]) * scale_o,
+                                    __uint_as_float(o[16 * v8 + 2 * j + 1]) * scale_o);
+              st_global_v8(orow + 16 * v8, pk);
+            }
+          } else {
+            uint4* orow4 = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int v4 = 0; v4 < 16; ++v4) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                pk[j] = pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * scale_o,
+                                    __uint_as_float(o[8 * v4 + 2 * j + 1]) * scale_o);
+              orow4[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
           }
         } else if (row_ok) {
           // e4m3 of O / out_scale: round to nearest even, saturated at 448
           const float qs = scale_o / *p.out_scale;
-          uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + out_off);
+          uint8_t* orow = static_cast<uint8_t*>(p.out) + out_off;
+          if (p.wide_out & 1) {
 #pragma unroll
-          for (int v16 = 0; v16 < 8; ++v16) {
-            uint32_t pk[4];
+            for (int v32 = 0; v32 < 4; ++v32) {  // 32 e4m3 per store
+              uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              pk[j] = pack_e4m3x4(__uint_as_float(o[16 * v16 + 4 * j]) * qs,
-                                  __uint_as_float(o[16 * v16 + 4 * j + 1]) * qs,
-                                  __uint_as_float(o[16 * v16 + 4 * j + 2]) * qs,
-                                  __uint_as_float(o[16 * v16 + 4 * j + 3]) * qs);
-            orow[v16] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              for (int j = 0; j < 8; ++j)
+                pk[j] = pack_e4m3x4(__uint_as_float(o[32 * v32 + 4 * j]) * qs,
+                                    __uint_as_float(o[32 * v32 + 4 * j + 1]) * qs,
+                                    __uint_as_float(o[32 * v32 + 4 * j + 2]) * qs,
+                                    __uint_as_float(o[32 * v32 + 4 * j + 3]) * qs);
+              st_global_v8(orow + 32 * v32, pk);
+            }
+          } else {
+            uint4* orow4 = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int v16 = 0; v16 < 8; ++v16) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                pk[j] = pack_e4m3x4(__uint_as_float(o[16 * v16 + 4 * j]) * qs,
+                                    __uint_as_float(o[16 * v16 + 4 * j + 1]) * qs,
+                                    __uint_as_float(o[16 * v16 + 4 * j + 2]) * qs,
+                                    __uint_as_float(o[16 * v16 + 4 * j + 3]) * qs);
+              orow4[v16] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
           }
         }
       } else if (row_ok && p.nsplit > 1) {

@@ -438,6 +438,15 @@ int dense_call(const DenseCall& c) {
     p.lse_part = reinterpret_cast<float*>(
         part + static_cast<size_t>(c.nsplit) * c.total_q * c.num_heads * kDv * sizeof(float));
   }
+  // 32-byte stores where every output row starts on a 32-byte boundary: the
+  // base, and the row and head strides in bytes (bf16 or e4m3 elements);
+  // the partials' rows are 512 bytes.
+  {
+    const long long esz = c.out_scale != nullptr ? 1 : 2;
+    const bool out32 = aligned(c.out, 32) && (p.out_rs * esz) % 32 == 0 &&
+                       (p.out_hs * esz) % 32 == 0;
+    p.wide_out = (out32 ? 1 : 0) | (p.o_part != nullptr && aligned(p.o_part, 32) ? 2 : 0);
+  }
   p.ws = ws;
   p.entries = entries;
   p.num_heads = c.num_heads;
@@ -820,6 +829,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv_latent, const int32_t* 
   p.num_rows = num_kv_rows;
   p.topk = topk;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+  p.wide_out = aligned(out, 32) ? 1 : 0;  // rows of 1024 bytes, halves of 512
   p.timeout_ns = wait_timeout_ns();
   sp::sparse_fwd_kernel<<<2 * num_tokens, sp::kThreads, sp::kSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(tm_q, p);

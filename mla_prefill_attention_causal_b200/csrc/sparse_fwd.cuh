@@ -87,6 +87,7 @@ struct Params {
   int num_rows;
   int topk;
   float scale_log2;
+  int wide_out;            // out is 32-byte aligned: every row half starts on a 32-byte boundary
   uint64_t timeout_ns;
 };
 
@@ -427,23 +428,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool seen = m_run != -INFINITY;  // some valid slot
       const float inv = seen ? 1.0f / l_run : 0.0f;
-      uint4* orow = reinterpret_cast<uint4*>(
-          p.out + (static_cast<size_t>(t) * p.num_heads + h) * kDv + half * kDvHalf);
+      __nv_bfloat16* orow = p.out + (static_cast<size_t>(t) * p.num_heads + h) * kDv + half * kDvHalf;
       const uint32_t tO = tmem + lane_off + kColO;
 #pragma unroll 1
       for (int q = 0; q < kDvHalf / 32; ++q) {
         uint32_t o[32];
         tmem_ld_x32_wait(tO + 32u * q, o);
         if (row_ok) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint32_t pk[4];
+          for (int j = 0; j < 16; ++j)  // no valid slot: O = 0 (TMEM O may be unwritten)
+            pk[j] = seen ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
+                                       __uint_as_float(o[2 * j + 1]) * inv)
+                         : 0u;
+          if (p.wide_out) {  // two 32-byte stores: whole L2 sectors
 #pragma unroll
-            for (int j = 0; j < 4; ++j)  // no valid slot: O = 0 (TMEM O may be unwritten)
-              pk[j] = seen ? pack_bf16x2(__uint_as_float(o[8 * v4 + 2 * j]) * inv,
-                                         __uint_as_float(o[8 * v4 + 2 * j + 1]) * inv)
-                           : 0u;
-            orow[4 * q + v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int w = 0; w < 2; ++w)
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                               orow + 32 * q + 16 * w),
+                           "r"(pk[8 * w]), "r"(pk[8 * w + 1]), "r"(pk[8 * w + 2]),
+                           "r"(pk[8 * w + 3]), "r"(pk[8 * w + 4]), "r"(pk[8 * w + 5]),
+                           "r"(pk[8 * w + 6]), "r"(pk[8 * w + 7])
+                           : "memory");
+          } else {
+            uint4* orow4 = reinterpret_cast<uint4*>(orow + 32 * q);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              orow4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
         }
       }

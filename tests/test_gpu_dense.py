@@ -462,3 +462,47 @@ def test_dims_call_with_the_default_geometry_is_the_plain_call():
                                         case["scale"], causal=True)
     o_p, l_p = run_dense(case)
     assert torch.equal(out, o_p) and torch.equal(lse, l_p)
+
+
+# -------------------------------------------------- output alignment (16 vs 32 bytes)
+def test_outputs_only_16_byte_aligned_give_the_same_bits():
+    """The epilogue stores 32-byte pieces where every output row is 32-byte
+    aligned and 16-byte pieces otherwise; outputs (bf16 and e4m3) and a
+    split-KV workspace that start 16 bytes past a 32-byte boundary must give
+    the bits of aligned ones."""
+    import mla_prefill_attention_causal_b200 as mla
+    case = syn.dense_case([513, 130, 1, 700], [513, 130, 1, 700], 4, seed=131)
+    q, k, v = dev_bf16(case["q"]), dev_bf16(case["k"]), dev_bf16(case["v"])
+    cq, ck = dev_i32(case["cu_q"]), dev_i32(case["cu_k"])
+    T, H = q.shape[0], q.shape[1]
+    args = (q, k, v, cq, ck, case["max_q"], case["max_k"], case["scale"])
+
+    def shifted(n_elems, dtype, shift_bytes):
+        esz = torch.empty((), dtype=dtype).element_size()
+        buf = torch.empty(n_elems + 64 // esz, dtype=dtype, device="cuda")
+        base = (-buf.data_ptr()) % 32 // esz + shift_bytes // esz  # 32-byte boundary + shift
+        return buf[base:base + n_elems]
+
+    o_a, l_a = mla.mla_prefill_fwd(*args, causal=True)
+    o_s = shifted(T * H * 128, torch.bfloat16, 16).view(T, H, 128)
+    assert o_s.data_ptr() % 32 == 16
+    mla.mla_prefill_fwd(*args, causal=True, out=o_s)
+    torch.cuda.synchronize()
+    assert torch.equal(o_s, o_a)
+
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    f_a, _ = mla.mla_prefill_fwd_ex(*args, causal=True, output_scale=sc)
+    f_s = shifted(T * H * 128, torch.uint8, 16).view(torch.float8_e4m3fn).view(T, H, 128)
+    assert f_s.data_ptr() % 32 == 16
+    mla.mla_prefill_fwd_ex(*args, causal=True, output_scale=sc, out=f_s)
+    torch.cuda.synchronize()
+    assert torch.equal(f_s.view(torch.uint8), f_a.view(torch.uint8))
+
+    ns = 3
+    wbytes = mla.splitkv_workspace_size(len(case["lens_q"]), T, H, ns)
+    s_a, sl_a = mla.mla_prefill_fwd_splitkv(*args, causal=True, num_splits=ns)
+    ws = shifted(wbytes, torch.uint8, 16)
+    assert ws.data_ptr() % 32 == 16
+    s_s, sl_s = mla.mla_prefill_fwd_splitkv(*args, causal=True, num_splits=ns, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(s_s, s_a) and torch.equal(sl_s, sl_a)

@@ -134,3 +134,23 @@ def test_workload_4096_tokens_full(cuda_ok, padded):
     out, lse = run_sparse(case)
     check_sparse_full(f"sparse 4096 x 128, top-k 2048{' padded' if padded else ''}",
                       case["q"], case["kv"], case["indices"], case["scale"], out, lse)
+
+
+def test_output_only_16_byte_aligned_gives_the_same_bits(cuda_ok):
+    """The epilogue stores 32-byte pieces when the output is 32-byte aligned
+    and 16-byte pieces otherwise; both give the same bits."""
+    import mla_prefill_attention_causal_b200 as mla
+    case = syn.sparse_case(num_tokens=9, num_heads=128, num_rows=700, topk=320, first_pos=600,
+                           seed=48)
+    q, kv = dev_bf16(case["q"]), dev_bf16(case["kv"])
+    idx = torch.from_numpy(case["indices"]).cuda()
+    a, la = mla.mla_sparse_prefill_fwd(q, kv, idx, case["scale"])
+    T, H = q.shape[0], q.shape[1]
+    n = T * H * 512
+    buf = torch.empty(n + 32, dtype=torch.bfloat16, device="cuda")
+    base = (-buf.data_ptr()) % 32 // 2 + 8  # 16 bytes past a 32-byte boundary
+    out = buf[base:base + n].view(T, H, 512)
+    assert out.data_ptr() % 32 == 16
+    b, lb = mla.mla_sparse_prefill_fwd(q, kv, idx, case["scale"], out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(b, a) and torch.equal(lb, la)

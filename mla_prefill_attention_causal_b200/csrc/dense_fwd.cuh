@@ -740,6 +740,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_cnt = 0;  // S blocks consumed (s_full parity)
     int o_cnt = 0;  // O-using tiles (o_full parity)
     bool ok = true;
+    // The second half of the previous tile's output row (64 bf16 as 32
+    // words), stored once the next tile's first P is published: the stores
+    // of a tile's epilogue otherwise delay that P, on which the MMA warp
+    // waits at the tile boundary (32-byte-aligned bf16 outputs only).
+    uint32_t dfr[32];
+    __nv_bfloat16* dfr_row = nullptr;
+    auto flush_dfr = [&]() {
+      if (dfr_row != nullptr) {
+#pragma unroll
+        for (int v8 = 0; v8 < 4; ++v8)
+          st_global_v8(dfr_row + 64 + 16 * v8, *reinterpret_cast<const uint32_t(*)[8]>(&dfr[8 * v8]));
+        dfr_row = nullptr;
+      }
+    };
     for (int k = 0; ok; ++k) {
       const int ts = tile_slot(k);
       ok = __all_sync(0xffffffffu, wait(smem_u32(&bars->tile_full[ts]), tile_par(k),
@@ -841,6 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(pbar_lead);
+        if (n == 0) flush_dfr();
       }
       if (!ok) break;
       const int e_lq = bars->tiles[ts].Lq;
@@ -855,6 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_release_cluster(lead(&bars->tile_empty[ts]));
 
+      flush_dfr();  // a tile without blocks for this sub-tile came in between
       // ------------------------------------------------------- epilogue
       // Denominator Z = l 2^m (+ 2^s for the head's sink s, in the same log2
       // units); O = O_acc 2^m / Z, LSE = log2(Z) ln 2.  Without a sink this
@@ -918,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + out_off;
           if (p.wide_out & 1) {
 #pragma unroll
-            for (int v8 = 0; v8 < 8; ++v8) {  // 16 bf16 per store
+            for (int v8 = 0; v8 < 4; ++v8) {  // 16 bf16 per store
               uint32_t pk[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -926,6 +942,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     __uint_as_float(o[16 * v8 + 2 * j + 1]) * scale_o);
               st_global_v8(orow + 16 * v8, pk);
             }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              dfr[j] = pack_bf16x2(__uint_as_float(o[64 + 2 * j]) * scale_o,
+                                   __uint_as_float(o[64 + 2 * j + 1]) * scale_o);
+            dfr_row = orow;
           } else {
             uint4* orow4 = reinterpret_cast<uint4*>(orow);
 #pragma unroll
@@ -987,6 +1008,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       else if (row_ok && p.lse != nullptr)
         p.lse[static_cast<size_t>(e_h) * p.total_q + e_q0 + r] = lse2 * 0.69314718055994530942f;
     }
+    flush_dfr();  // the last tile's deferred half
   }
 
   // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still
